@@ -1,0 +1,6 @@
+"""fp64 CPU oracle for the KDA forward pass.
+
+Test infrastructure: only the tests, ``__graft_entry__.smoke()`` and the bench's CPU-baseline
+leg use it.  It never imports the CUDA package, and the CUDA package never imports it.
+"""
+from .oracle import forward, decode_step, max_threads, RULE_DELTA, RULE_ADDITIVE  # noqa: F401
