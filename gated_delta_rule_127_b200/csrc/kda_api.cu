@@ -1,0 +1,149 @@
+// kda_api.cu -- the C ABI of libkda: host-side validation, dispatch to the kernels, status words.
+//
+// Nothing here computes any part of the operator; it checks arguments, picks the kernel and
+// launches it on the caller's stream.
+#include <mutex>
+
+#include "kda.h"
+#include "kda_internal.h"
+
+namespace kda {
+
+// One sticky status word per device; kernels OR KDA_DEVFLAG_* bits into it.
+__device__ unsigned int g_device_flags = 0u;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_flag_mutex;
+unsigned int* g_flag_addr[kMaxDevices] = {};
+
+// Device address of g_device_flags for the current device (looked up once per device).
+cudaError_t device_flags_ptr(unsigned int** out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_flag_mutex);
+    if (!g_flag_addr[dev]) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_device_flags);
+        if (err != cudaSuccess) return err;
+        g_flag_addr[dev] = static_cast<unsigned int*>(p);
+    }
+    *out = g_flag_addr[dev];
+    return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool valid_dtype(kda_dtype d) { return d == KDA_BF16 || d == KDA_FP32; }
+size_t dtype_size(kda_dtype d) { return d == KDA_FP32 ? 4 : 2; }
+bool supported_dim(int d) { return d == 64 || d == 128; }
+
+}  // namespace
+}  // namespace kda
+
+extern "C" {
+
+size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int dk, int dv, int chunk_size) {
+    (void)chunk_size;
+    if (T_total < 0 || N <= 0 || H <= 0) return 0;
+    return kda::chunk_tc_workspace_size(T_total, N, H, dk, dv);
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
+                         const void* beta, const float* initial_state, const int32_t* cu_seqlens,
+                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                         float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+    using namespace kda;
+    if (T_total < 0 || N <= 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk_size <= 0)
+        return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
+        return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(dk) || !supported_dim(dv) || chunk_size != 64) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens && (T_total % N) != 0) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)N * H * (dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (T_total > 0) {
+        if (!q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
+            return KDA_ERR_INVALID_ARG;
+        if (!aligned_to(beta, dtype_size(dtype_gate))) return KDA_ERR_INVALID_ARG;
+    }
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_chunk_fwd_workspace_size(T_total, N, H, dk, dv, chunk_size);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+        return KDA_ERR_INVALID_ARG;
+
+    ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
+    a.T_total = T_total; a.N = N; a.H = H; a.dk = dk; a.dv = dv;
+    a.dtype_qkv = dtype_qkv; a.dtype_gate = dtype_gate; a.dtype_o = dtype_o;
+    a.o = o; a.final_state = final_state; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    a.stream = static_cast<cudaStream_t>(stream);
+    if (device_flags_ptr(&a.flags) != cudaSuccess) return KDA_ERR_CUDA;
+
+    const cudaError_t err = chunk_tc_supported(a) ? launch_chunk_tc(a) : launch_chunk_simt(a);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
+                           const void* beta, float* state, int B, int H, int dk, int dv,
+                           kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                           void* stream) {
+    using namespace kda;
+    if (B < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
+        return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(dk) || !supported_dim(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (B == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(state) || !aligned_to(q, dtype_size(dtype_qkv)) || !aligned_to(k, dtype_size(dtype_qkv)) ||
+        !aligned_to(v, dtype_size(dtype_qkv)) || !aligned_to(log_alpha, dtype_size(dtype_gate)) ||
+        !aligned_to(beta, dtype_size(dtype_gate)) || !aligned_to(o, dtype_size(dtype_o)))
+        return KDA_ERR_INVALID_ARG;
+
+    DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.state = state;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+    a.dtype_qkv = dtype_qkv; a.dtype_gate = dtype_gate; a.dtype_o = dtype_o; a.o = o;
+    a.stream = static_cast<cudaStream_t>(stream);
+    a.flags = nullptr;
+    return launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_get_device_status(void* stream, uint32_t* flags) {
+    using namespace kda;
+    if (flags) *flags = 0;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned int* addr = nullptr;
+    if (device_flags_ptr(&addr) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned int value = 0, zero = 0;
+    if (cudaMemcpy(&value, addr, sizeof(value), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    if (value && cudaMemcpy(addr, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (flags) *flags = value;
+    if (value & KDA_DEVFLAG_TIMEOUT) return KDA_ERR_TIMEOUT;
+    return value ? KDA_ERR_DEVICE_CHECK : KDA_OK;
+}
+
+const char* kda_status_string(kda_status status) {
+    switch (status) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_INVALID_ARG: return "invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case KDA_ERR_CUDA: return "CUDA error";
+        case KDA_ERR_TIMEOUT: return "a bounded device wait timed out";
+        case KDA_ERR_DEVICE_CHECK: return "a device-side check failed";
+    }
+    return "unknown status";
+}
+
+uint32_t kda_version(void) { return (1u << 16) | 0u; }
+
+}  // extern "C"

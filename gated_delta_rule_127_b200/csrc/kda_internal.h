@@ -1,0 +1,51 @@
+// kda_internal.h -- launchers shared between the host API (kda_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+struct ChunkArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* log_alpha;
+    const void* beta;
+    const float* initial_state;
+    const int32_t* cu_seqlens;  // may be NULL: equal lengths T_total / N
+    int64_t T_total;
+    int N, H, dk, dv;
+    kda_dtype dtype_qkv, dtype_gate, dtype_o;
+    void* o;
+    float* final_state;
+    void* workspace;
+    size_t workspace_bytes;
+    unsigned int* flags;  // device address of the sticky flag word
+    cudaStream_t stream;
+};
+
+struct DecodeArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* log_alpha;
+    const void* beta;
+    float* state;
+    int B, H, dk, dv;
+    kda_dtype dtype_qkv, dtype_gate, dtype_o;
+    void* o;
+    unsigned int* flags;
+    cudaStream_t stream;
+};
+
+// Each launcher returns cudaSuccess or the launch error.
+cudaError_t launch_decode(const DecodeArgs& a);
+cudaError_t launch_chunk_simt(const ChunkArgs& a);
+cudaError_t launch_chunk_tc(const ChunkArgs& a);
+bool chunk_tc_supported(const ChunkArgs& a);
+size_t chunk_tc_workspace_size(int64_t T_total, int N, int H, int dk, int dv);
+
+}  // namespace kda

@@ -1,0 +1,143 @@
+/*
+ * kda.h -- C ABI of libkda, the Kimi Delta Attention (KDA) forward pass on B200 (sm_100a).
+ *
+ * The operator.  Per (sequence, head), with state S in R^{dk x dv}:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,    o_t = S_t^T q_t,
+ *
+ * alpha_t = exp(log_alpha_t) in (0,1)^{dk} (a channel-wise decay on the key axis), beta_t in (0,1)
+ * a scalar per token and head.  Source: "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)"
+ * (GeekNews topic 31936), section "Kimi Delta Attention의 세밀한 메모리 제어" (Gated DeltaNet's
+ * scalar forget gate refined to one rate per feature channel) building on section "선형 어텐션에서
+ * Gated DeltaNet까지" (delta rule, scalar gate); and "From GPT-2 to Kimi K3, Explained", section
+ * "Kimi Linear (KDA) -- 채널별 세밀한 게이팅" (alpha becomes Diag(alpha)).
+ * Readings taken where the pages leave a step open: the delta read uses the decayed state
+ * Diag(alpha_t) S_{t-1}; the output is read after the write; there is no query scale.
+ *
+ * Conventions for every entry point:
+ *   - Every tensor pointer is caller-owned DEVICE memory (cudaMalloc / PyTorch), densely packed
+ *     row-major in the layout given, 16-byte aligned.  The library keeps no pointer after a call
+ *     returns and allocates no device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Calls are
+ *     asynchronous on that stream: a returned KDA_OK means "validated and launched".
+ *   - Arguments are validated on the host before any launch; an invalid argument returns a status
+ *     and launches nothing.  Problems only the device can see (the contents of cu_seqlens, a decay
+ *     range the tensor-core path cannot represent) set sticky flags that kda_get_device_status
+ *     reads.  Nothing traps or asserts on the device.
+ *   - dtypes: q/k/v share `dtype_qkv`; log_alpha/beta share `dtype_gate`; o has `dtype_o`.
+ *     The recurrent state is always fp32.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, workspace too small */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented: dk, dv not in {64,128}, chunk != 64 */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 4,       /* a bounded device wait gave up (see kda_get_device_status) */
+    KDA_ERR_DEVICE_CHECK = 5   /* a device-side argument check failed (see kda_get_device_status) */
+} kda_status;
+
+typedef enum { KDA_BF16 = 0, KDA_FP32 = 1 } kda_dtype;
+
+/* Sticky device flags returned by kda_get_device_status (bitwise OR). */
+#define KDA_DEVFLAG_CU_SEQLENS 0x1u   /* cu_seqlens[0] != 0, decreasing, or cu_seqlens[N] != T_total;
+                                         the offending sequences were skipped */
+#define KDA_DEVFLAG_DECAY_RANGE 0x2u  /* within some 64-token chunk the cumulative log-decay moved by
+                                         more than 80 (nats) between the chunk's middle row and its
+                                         first or last row; the bf16 tensor-core path's outputs for
+                                         that chunk are not reliable (the fp32 path is exact there) */
+#define KDA_DEVFLAG_TIMEOUT 0x4u      /* a bounded inter-CTA wait gave up */
+
+/*
+ * Workspace bytes kda_chunk_fwd needs for these sizes (0 is a valid answer).
+ * T_total: packed tokens; N: sequences.  Pure host function, no CUDA call.
+ */
+KDA_API size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int dk, int dv, int chunk_size);
+
+/*
+ * Chunkwise-parallel KDA prefill over a packed batch of N variable-length sequences.
+ *
+ * Passage: "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "청크 단위 병렬
+ * 알고리듬": fixed-length chunks, each starting from the previous chunk's final state; the WY
+ * representation packs the chunk's rank-1 updates; the UT transform; the lower-triangular inverse
+ * by forward substitution; chunk-level state recurrence plus intra-chunk parallel output with the
+ * intra-chunk work arranged as matrix multiplies for the tensor cores.
+ *
+ *   q, k        [T_total, H, dk]  dtype_qkv        queries, keys (callers usually L2-normalise)
+ *   v           [T_total, H, dv]  dtype_qkv        values
+ *   log_alpha   [T_total, H, dk]  dtype_gate       natural log of the decay, <= 0
+ *   beta        [T_total, H]      dtype_gate       write strength
+ *   initial_state [N, H, dk, dv]  fp32 or NULL     NULL = zero initial state
+ *   cu_seqlens  [N+1] int32 (device) or NULL       token offsets, cu_seqlens[0] = 0, non-decreasing,
+ *                                                  cu_seqlens[N] = T_total.  NULL = N sequences of
+ *                                                  T_total / N tokens each (T_total % N must be 0).
+ *                                                  Contents are checked on the device only.
+ *   T_total >= 0, N >= 1, H >= 1, dk, dv in {64, 128}, chunk_size == 64
+ *   o           [T_total, H, dv]  dtype_o          output (may not alias an input)
+ *   final_state [N, H, dk, dv]    fp32 or NULL     NULL = not written; may alias initial_state
+ *   workspace   device scratch of workspace_bytes >= kda_chunk_fwd_workspace_size(...), or NULL
+ *               when that size is 0.
+ *
+ * Path: dtype_qkv == KDA_FP32 runs the fp32 CUDA-core path (every product in fp32); KDA_BF16 with
+ * dk = dv = 128 runs the tensor-core path (bf16 operands, fp32 accumulation and fp32 state).
+ */
+KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
+                         const void* log_alpha, const void* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
+                         void* o, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One recurrent decode step for B sequences (one new token each), state updated in place.
+ *
+ * Passage: "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "NoPE 적용과 평가
+ * 결과" (decoding keeps a fixed-size recurrent state instead of a growing KV cache; time per output
+ * token), with the step of section "Kimi Delta Attention의 세밀한 메모리 제어".
+ *
+ *   q, k        [B, H, dk]  dtype_qkv;  v [B, H, dv] dtype_qkv
+ *   log_alpha   [B, H, dk]  dtype_gate; beta [B, H] dtype_gate
+ *   state       [B, H, dk, dv] fp32, read and overwritten with the new state
+ *   o           [B, H, dv]  dtype_o
+ *   B >= 0 (0 launches nothing), H >= 1, dk, dv in {64, 128}
+ */
+KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v,
+                           const void* log_alpha, const void* beta, float* state,
+                           int B, int H, int dk, int dv,
+                           kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
+                           void* o, void* stream);
+
+/*
+ * Waits for `stream`, then reads and clears the sticky device flags (KDA_DEVFLAG_*) of the current
+ * device into *flags (may be NULL).  Returns KDA_OK if no flag was set, KDA_ERR_TIMEOUT if the
+ * timeout flag was set, KDA_ERR_DEVICE_CHECK for any other flag, KDA_ERR_CUDA on a CUDA error.
+ */
+KDA_API kda_status kda_get_device_status(void* stream, uint32_t* flags);
+
+/* Static English text for a status code; never NULL. */
+KDA_API const char* kda_status_string(kda_status status);
+
+/* Library ABI version, (major << 16) | minor. */
+KDA_API uint32_t kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,96 @@
+"""The C ABI without a GPU: the library loads, exports every entry point include/kda.h declares, and
+rejects invalid arguments on the host before any CUDA call (no compute call is made here)."""
+import ctypes
+
+import pytest
+
+from gated_delta_rule_127_b200 import build as kbuild
+from gated_delta_rule_127_b200 import kda
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def test_header_declares_the_entry_points():
+    names = set(kda.header_symbols())
+    assert {"kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_get_device_status",
+            "kda_status_string", "kda_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in kda.header_symbols():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version(lib):
+    assert kda.kda_status_string(kda.KDA_OK) == "ok"
+    for st in range(1, 6):
+        assert kda.kda_status_string(st) not in ("", "ok", "unknown status")
+    assert kda.kda_status_string(99) == "unknown status"
+    assert kda.kda_version() >> 16 == 1
+
+
+FAKE = 1 << 20  # 16-byte aligned fake device address: never dereferenced, validation fails first
+
+
+def _chunk(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, cu=None, T=128, N=1, H=2, dk=128, dv=128,
+             chunk=64, dq=kda.KDA_BF16, dg=kda.KDA_FP32, do=kda.KDA_FP32, o=FAKE, sf=None, ws=None, wsb=0)
+    a.update(kw)
+    return lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["cu"], a["T"], a["N"], a["H"],
+                             a["dk"], a["dv"], a["chunk"], a["dq"], a["dg"], a["do"], a["o"], a["sf"], a["ws"],
+                             a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=128), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dv=256), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=100, N=3), kda.KDA_ERR_INVALID_ARG),          # equal lengths need T % N == 0
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(o=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(k=FAKE + 8), kda.KDA_ERR_INVALID_ARG),           # misaligned
+    (dict(s0=FAKE + 4), kda.KDA_ERR_INVALID_ARG),
+    (dict(cu=FAKE + 2), kda.KDA_ERR_INVALID_ARG),
+    (dict(dq=7), kda.KDA_ERR_INVALID_ARG),
+    (dict(do=-1), kda.KDA_ERR_INVALID_ARG),
+])
+def test_chunk_fwd_rejects_on_host(lib, kw, expect):
+    assert _chunk(lib, **kw) == expect
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S=FAKE, B=4, H=2, dk=128, dv=128, dq=kda.KDA_BF16,
+             dg=kda.KDA_FP32, do=kda.KDA_FP32, o=FAKE)
+    a.update(kw)
+    return lib.kda_decode_step(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S"], a["B"], a["H"], a["dk"],
+                               a["dv"], a["dq"], a["dg"], a["do"], a["o"], None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(B=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(S=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(S=FAKE + 4), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=FAKE + 1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dg=5), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=0), kda.KDA_OK),                                  # nothing to do, nothing launched
+])
+def test_decode_step_rejects_on_host(lib, kw, expect):
+    assert _decode(lib, **kw) == expect
+
+
+def test_workspace_size_is_a_pure_host_function(lib):
+    assert kda.kda_chunk_fwd_workspace_size(0, 1, 1, 128, 128) >= 0
+    assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) >= 0
+    assert lib.kda_chunk_fwd_workspace_size(-1, 1, 1, 128, 128, 64) == 0

@@ -1,0 +1,198 @@
+"""GPU parity of kda_chunk_fwd against the fp64 oracle, called through the C ABI.
+
+Small and mid-size cases compare every output element and every state element; the full-size
+workloads compare every element of sampled (sequence, head) units, in the launch configuration the
+bench times.  Tolerances are those stated in tests/parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_127_b200 import inputs as gen
+from gated_delta_rule_127_b200 import kda
+from parity import TOL, o_err, oracle_full, oracle_units, s_err, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from gated_delta_rule_127_b200 import build
+    build.build()
+    kda.load_library()
+
+
+def _run(inp, dtype_o=torch.float32):
+    o, sf = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, inp.cu_seqlens,
+                              dtype_o=dtype_o)
+    st, flags = kda.kda_get_device_status()
+    assert st == kda.KDA_OK and flags == 0, (st, flags)
+    return o, sf
+
+
+def _check_full(inp, dtype):
+    o, sf = _run(inp)
+    o_ref, s_ref = oracle_full(inp)
+    eo, es = o_err(to_np(o), o_ref), s_err(to_np(sf), s_ref)
+    tol_o, tol_s = TOL[dtype]
+    assert np.isfinite(eo) and eo <= tol_o, eo
+    assert np.isfinite(es) and es <= tol_s, es
+    return eo, es
+
+
+def test_tiny_fp32_workload():
+    inp = gen.make_workload("tiny_fp32", device=DEV)
+    _check_full(inp, torch.float32)
+
+
+def test_prefill_b2_h4_t2048_workload():
+    inp = gen.make_workload("prefill_b2_h4_t2048", device=DEV)
+    _check_full(inp, torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_ragged_varlen(dtype, dk, dv):
+    lengths = [1, 63, 64, 65, 130, 0, 200, 7]
+    inp = gen.make_prefill(lengths, 3, dk, dv, dtype=dtype, init_state=True, seed=11, device=DEV)
+    _check_full(inp, dtype)
+
+
+def test_bf16_gates():
+    inp = gen.make_prefill([300, 77], 2, 128, 128, dtype=torch.bfloat16, gate_dtype=torch.bfloat16,
+                           init_state=True, seed=12, device=DEV)
+    _check_full(inp, torch.bfloat16)
+
+
+def test_zero_initial_state_and_no_final_state():
+    inp = gen.make_prefill([192], 2, 128, 128, dtype=torch.bfloat16, init_state=False, seed=13, device=DEV)
+    o, sf = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, inp.cu_seqlens,
+                              dtype_o=torch.float32, output_final_state=False)
+    assert sf is None
+    o_ref, _ = oracle_full(inp)
+    assert o_err(to_np(o), o_ref) <= TOL[torch.bfloat16][0]
+
+
+def test_bf16_output_is_the_rounded_fp32_output():
+    inp = gen.make_prefill([256, 100], 2, 128, 128, dtype=torch.bfloat16, seed=14, device=DEV)
+    o32, _ = _run(inp, torch.float32)
+    o16, _ = _run(inp, torch.bfloat16)
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+
+
+def test_empty_batch_passes_state_through():
+    inp = gen.make_prefill([0, 0], 2, 128, 128, dtype=torch.bfloat16, init_state=True, seed=15, device=DEV)
+    o, sf = _run(inp)
+    assert o.numel() == 0
+    assert torch.equal(sf, inp.initial_state)
+
+
+def test_final_state_may_alias_initial_state():
+    inp = gen.make_prefill([150, 64], 2, 128, 128, dtype=torch.bfloat16, init_state=True, seed=16, device=DEV)
+    o_ref, s_ref = _run(inp)
+    state = inp.initial_state.clone()
+    o, sf = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, state, inp.cu_seqlens,
+                              final_state=state, dtype_o=torch.float32)
+    assert sf.data_ptr() == state.data_ptr()
+    assert torch.equal(o, o_ref) and torch.equal(state, s_ref)
+
+
+def test_equal_lengths_without_cu_seqlens():
+    inp = gen.make_prefill([128, 128, 128], 2, 128, 128, dtype=torch.bfloat16, seed=17, device=DEV)
+    o1, s1 = _run(inp)
+    o2, s2 = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, None,
+                               num_seqs=3, dtype_o=torch.float32)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_invalid_cu_seqlens_sets_device_flag():
+    inp = gen.make_prefill([100, 100], 1, 128, 128, dtype=torch.bfloat16, seed=18, device=DEV)
+    bad = torch.tensor([0, 150, 120], dtype=torch.int32, device=DEV)  # decreasing
+    kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, bad,
+                      dtype_o=torch.float32)
+    st, flags = kda.kda_get_device_status()
+    assert st == kda.KDA_ERR_DEVICE_CHECK and flags & kda.KDA_DEVFLAG_CU_SEQLENS
+    assert kda.kda_get_device_status() == (kda.KDA_OK, 0)  # reading cleared it
+
+
+def test_host_rejects_unsupported_chunk_size():
+    inp = gen.make_prefill([64], 1, 128, 128, dtype=torch.bfloat16, seed=19, device=DEV)
+    with pytest.raises(kda.KdaError) as e:
+        kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, chunk_size=32)
+    assert e.value.status == kda.KDA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- properties of the true result
+
+def test_continuation_equals_one_pass():
+    inp = gen.make_prefill([1000], 2, 128, 128, dtype=torch.bfloat16, seed=20, device=DEV)
+    o, sf = _run(inp)
+    cut = 437
+    o1, s1 = kda.kda_chunk_fwd(inp.q[:cut], inp.k[:cut], inp.v[:cut], inp.log_alpha[:cut], inp.beta[:cut],
+                               inp.initial_state, dtype_o=torch.float32)
+    o2, s2 = kda.kda_chunk_fwd(inp.q[cut:].contiguous(), inp.k[cut:].contiguous(), inp.v[cut:].contiguous(),
+                               inp.log_alpha[cut:].contiguous(), inp.beta[cut:].contiguous(), s1,
+                               dtype_o=torch.float32)
+    tol_o, tol_s = TOL[torch.bfloat16]
+    assert o_err(to_np(torch.cat([o1, o2])), to_np(o)) <= tol_o
+    assert s_err(to_np(s2), to_np(sf)) <= tol_s
+
+
+def test_packed_equals_separate_calls():
+    lengths = [70, 129, 1, 300]
+    inp = gen.make_prefill(lengths, 2, 128, 128, dtype=torch.bfloat16, seed=21, device=DEV)
+    o, sf = _run(inp)
+    a = 0
+    for n, L in enumerate(lengths):
+        on, sn = kda.kda_chunk_fwd(inp.q[a:a + L], inp.k[a:a + L], inp.v[a:a + L], inp.log_alpha[a:a + L],
+                                   inp.beta[a:a + L], inp.initial_state[n:n + 1].contiguous(),
+                                   dtype_o=torch.float32)
+        assert torch.equal(on, o[a:a + L]) and torch.equal(sn[0], sf[n])
+        a += L
+
+
+def test_prefill_equals_repeated_decode():
+    inp = gen.make_prefill([150], 2, 128, 128, dtype=torch.bfloat16, seed=22, device=DEV)
+    o, sf = _run(inp)
+    state = inp.initial_state.clone()
+    outs = []
+    for t in range(150):
+        outs.append(kda.kda_decode_step(inp.q[t:t + 1], inp.k[t:t + 1], inp.v[t:t + 1], inp.log_alpha[t:t + 1],
+                                        inp.beta[t:t + 1], state, dtype_o=torch.float32))
+    tol_o, tol_s = TOL[torch.bfloat16]
+    assert o_err(to_np(torch.cat(outs)), to_np(o)) <= tol_o
+    assert s_err(to_np(state), to_np(sf)) <= tol_s
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled units
+
+def _check_units(inp, units, o, sf, dtype):
+    ref = oracle_units(inp, units)
+    o_cmp, o_ref, s_cmp, s_ref = [], [], [], []
+    for (n, h), ((a, b), ou, Su) in ref.items():
+        o_cmp.append(to_np(o[a:b, h]))
+        o_ref.append(ou)
+        s_cmp.append(to_np(sf[n, h]))
+        s_ref.append(Su)
+    eo = o_err(np.concatenate(o_cmp), np.concatenate(o_ref))
+    es = s_err(np.stack(s_cmp), np.stack(s_ref))
+    tol_o, tol_s = TOL[dtype]
+    assert eo <= tol_o and es <= tol_s, (eo, es)
+    assert torch.isfinite(o).all() and torch.isfinite(sf).all()
+
+
+@pytest.mark.slow
+def test_prefill_b1_h32_t32768_sampled():
+    inp = gen.make_workload("prefill_b1_h32_t32768", device=DEV)
+    o, sf = _run(inp)
+    _check_units(inp, [(0, 0), (0, 13), (0, 31)], o, sf, torch.bfloat16)
+
+
+@pytest.mark.slow
+def test_varlen_n16_h32_sampled():
+    inp = gen.make_workload("varlen_n16_h32", device=DEV)
+    o, sf = _run(inp)
+    L = inp.lengths
+    units = [(int(np.argmin(L)), 0), (int(np.argmax(L)), 31), (5, 7), (15, 16)]
+    _check_units(inp, units, o, sf, torch.bfloat16)
