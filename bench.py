@@ -40,7 +40,7 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 64 * (3 * 128 + 2 * 128)
 # Decode: the fp32 state read and written once, plus q, k, v bf16, log_alpha fp32, beta fp32, o bf16.
 DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
-PREFILL_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_chunk_tc.cu",
+PREFILL_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_chunk_tc.cu", "gated_delta_rule_127_b200/csrc/kda_sm100.cuh",
                           "gated_delta_rule_127_b200/csrc/kda_chunk_simt.cu"]
 DECODE_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_decode.cu"]
 
@@ -102,7 +102,7 @@ class ClockSampler:
         self.proc = None
         self.marks = []
         try:
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            bus = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
         except Exception:
             bus = None
         self.bus = bus
@@ -387,9 +387,9 @@ def run_ours(args):
         if not args.no_cpu_baseline and world == 1:
             cores = len(os.sched_getaffinity(0))
             n_units = max(1, min(H, cores))
-            rate, threads, secs = oracle_sample_rate(inp, n_units, 16384)
+            rate, threads, secs = oracle_sample_rate(inp, n_units, 32768)
             cpu = {"value": rate / H, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                   "sample": f"{n_units} (head) units x first 16384 tokens of {PREFILL} ({secs:.1f} s wall, "
+                   "sample": f"{n_units} (head) units x all 32768 tokens of {PREFILL} ({secs:.1f} s wall, "
                              f"fp64 sequential recurrence, OpenMP over units)"}
         line = {
             "metric": "KDA chunked-prefill tokens/s (decode-step state GB/s in 'decode')",
