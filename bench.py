@@ -53,6 +53,10 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--only", choices=["prefill", "decode"], default=None,
+                   help="profiling aid: run only one leg (with --no-e2e --no-cpu-baseline)")
+    p.add_argument("--prefill-tokens", type=int, default=None,
+                   help="profiling aid: prefill sequence length instead of the workload's 32768")
     return p.parse_args(argv)
 
 
@@ -278,7 +282,11 @@ def run_ours(args):
 
     wp = gen.WORKLOADS[PREFILL]
     wd = gen.WORKLOADS[DECODE]
-    inp = gen.make_workload(PREFILL, seed=rank, device=device)
+    if args.prefill_tokens is None:
+        inp = gen.make_workload(PREFILL, seed=rank, device=device)
+    else:  # same distributions, shorter sequence (profiling aid only)
+        inp = gen.make_prefill([args.prefill_tokens], wp["H"], wp["dk"], wp["dv"], dtype=wp["dtype"],
+                               init_state=wp["init_state"], seed=rank, device=device)
     T, H = inp.T_total, inp.H
     o = torch.empty((T, H, inp.dv), dtype=torch.bfloat16, device=device)
     sf = torch.empty((inp.N, H, inp.dk, inp.dv), dtype=torch.float32, device=device)
@@ -293,10 +301,14 @@ def run_ours(args):
     stream = torch.cuda.current_stream(device)
 
     def prefill():
+        if args.only == "decode":
+            return
         kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, inp.cu_seqlens,
                           o=o, final_state=sf, workspace=ws, stream=stream)
 
     def decode(i):
+        if args.only == "prefill":
+            return
         x = dec_inputs[i % n_dec_inputs]
         kda.kda_decode_step(x.q, x.k, x.v, x.log_alpha, x.beta, state, o=od, stream=stream)
 

@@ -34,8 +34,15 @@
 // about 5e-3.  K-major operands use the 128-byte swizzle; MN-major tf32 operands must use the
 // 128-byte layout with 32-byte atoms.
 //
-// One CTA of 128 threads owns one (sequence, head, 32-column slice of dv) and walks its chunks in
-// order.  Thread c owns key channel c in the elementwise stage and row c of the state.
+// One CTA of 256 threads owns one (sequence, head, 32-column slice of dv) and walks its chunks in
+// order.  The raw q, k, log_alpha and v tiles of the next chunk are brought into shared memory by
+// TMA while the current chunk computes.  Thread t owns key channel / state row c = t % 128 and
+// half h2 = t / 128 of that channel's rows in the elementwise stage and of the state row's columns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_sm100.cuh"
@@ -49,29 +56,36 @@ constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DV = 128;
 constexpr int DVS = 32;
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;
 constexpr int TP = 65;              // padded row stride of the fp32 A and T tiles
 constexpr float kAnchorLimit = 80.f;
 constexpr uint32_t kWaitPolls = 1u << 26;
 
-// Shared memory (byte offsets from a 1024-aligned base).  "K-major" tiles use sw128_off, "MN-major"
-// tiles sw32b_off; rows = rows per 32-column block.
-constexpr uint32_t OFF_KQ = 0;         // [K+ ; Q+]  K-major 128 x 128 (64 KB); dead after batch 1, then:
-constexpr uint32_t OFF_A = 0;          //   A  fp32 [64][65]
-constexpr uint32_t OFF_TF = 16640;     //   T  fp32 [64][65]
-constexpr uint32_t OFF_T = 33792;      //   T' K-major 64 x 64 (16 KB)
-constexpr uint32_t OFF_Y = 50176;      //   768 floats of block-inverse scratch
-constexpr uint32_t OFF_KM = 65536;     // K-  K-major 64 x 128 (32 KB); dead after batch 1, then:
-constexpr uint32_t OFF_P = 65536;      //   P  K-major 64 x 64 (16 KB)
-constexpr uint32_t OFF_Z = 81920;      //   Z  MN-major 64 x 32 (8 KB)
-constexpr uint32_t OFF_KMM = 98304;    // K-  MN-major (K-rows i, M = channels c) 64 x 128 (32 KB)
+// Shared memory (byte offsets from a 1024-aligned base).  K-major tiles use sw128_off (16-byte
+// chunks), MN-major tiles sw32b_off (32-byte chunks); "rows" = rows per 32-column block.  The three
+// operand tiles of the elementwise stage are stored transposed (row = key channel c), so each
+// thread writes whole rows of its own channel with 16-byte stores.
+constexpr uint32_t OFF_KQ = 0;         // [K+ | Q+]^T  MN-major, K-rows c (128) x M-cols r (128): 64 KB
+constexpr uint32_t OFF_A = 0;          //   after batch 1: A  fp32 [64][65]
+constexpr uint32_t OFF_TF = 16640;     //                  T  fp32 [64][65]
+constexpr uint32_t OFF_T = 33792;      //                  T' K-major 64 x 64 (16 KB)
+constexpr uint32_t OFF_Y = 50176;      //                  1024 floats of block-inverse scratch
+constexpr uint32_t OFF_KM = 65536;     // (K-)^T  MN-major, K-rows c (128) x N-cols i (64): 32 KB
+constexpr uint32_t OFF_P = 65536;      //   after batch 1: P  K-major 64 x 64 (16 KB)
+constexpr uint32_t OFF_Z = 81920;      //                  Z  MN-major 64 x 32 (8 KB)
+constexpr uint32_t OFF_KMT = 98304;    // (K-)^T  K-major, rows c (128) x K-cols i (64): 32 KB
 constexpr uint32_t OFF_S = 131072;     // S'  MN-major 128 x 32 (16 KB)
-constexpr uint32_t OFF_V = 147456;     // V   MN-major 64 x 32 (8 KB)
-constexpr uint32_t OFF_D = 155648;     // Delta MN-major 64 x 32 (8 KB)
-constexpr uint32_t OFF_BETA = 163840;  // 64 floats
-constexpr uint32_t OFF_BAR = 164096;   // mbarrier (8 bytes)
-constexpr uint32_t OFF_SLOT = 164104;  // tensor-memory base address
-constexpr uint32_t SMEM_USED = 164112;
+constexpr uint32_t OFF_VD = 147456;    // V, then Delta: MN-major 64 x 32 (8 KB)
+constexpr uint32_t OFF_SK = 155648;    // TMA staging: k   bf16 [64][128]
+constexpr uint32_t OFF_SQ = 172032;    //              q   bf16 [64][128]
+constexpr uint32_t OFF_SLA = 188416;   //              log_alpha [64][128] (fp32 or bf16)
+constexpr uint32_t OFF_SV = 221184;    //              v   bf16 [64][32]
+constexpr uint32_t OFF_BETA = 225280;  // 64 floats
+constexpr uint32_t OFF_XCH = 225536;   // 3 x 128 floats: half-column sums, g at row 32, g at row 63
+constexpr uint32_t OFF_BAR = 227072;   // mbarrier: MMA completion
+constexpr uint32_t OFF_TBAR = 227080;  // mbarrier: TMA completion
+constexpr uint32_t OFF_SLOT = 227088;  // tensor-memory base address
+constexpr uint32_t SMEM_USED = 227096;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 
 // Tensor-memory columns (fp32).  Batch 2 and 3 reuse the columns batch 1 results were read from.
@@ -95,56 +109,103 @@ __device__ __forceinline__ void st_mn8(unsigned char* base, uint32_t off, int k_
     d[1] = make_float4(to_tf32(x[4]), to_tf32(x[5]), to_tf32(x[6]), to_tf32(x[7]));
 }
 
-// T = (I + A)^{-1}, A strictly lower 64 x 64 (fp32, row stride TP): forward substitution inside
-// the four 16 x 16 diagonal blocks, then block rows T_RI = -T_RR sum_{I<=J<R} A_RJ T_JI.
+// Four consecutive elements (col multiple of 4) of one row of a K-major tile, rounded to tf32.
+__device__ __forceinline__ void st_sw4(unsigned char* base, uint32_t off, int row, int col, int rows,
+                                       float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(base + off + sw128_off(row, col, rows)) =
+        make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
+}
+
+// T = (I + A)^{-1} for strictly lower A (64 x 64, fp32, row stride TP), by forward substitution:
+// inside each 16 x 16 diagonal block column by column (registers), then doubling the solved
+// block: for [T11 0; T21 T22] with T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1},
+// T21 = -T22 (A21 T11) -- first for 16 -> 32 (two blocks at once), then 32 -> 64.
 __device__ void unit_lower_inverse(const float* am, float* tm, float* y) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int idx = tid; idx < C * C; idx += THREADS) {
-        const int r = idx >> 6, j = idx & 63;
-        if ((j >> 4) > (r >> 4)) tm[r * TP + j] = 0.f;
-    }
-    if (lane < 16) {
-        const int b = warp * 16, j = lane;
-        for (int r = 0; r < 16; ++r) {
-            float acc = (r == j) ? 1.f : 0.f;
-            for (int i = j; i < r; ++i) acc -= am[(b + r) * TP + b + i] * tm[(b + i) * TP + b + j];
-            tm[(b + r) * TP + b + j] = (r >= j) ? acc : 0.f;
+    if (warp < 4) {
+        if (lane < 16) {
+            const int b = warp * 16, j = lane;
+            float t[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int i = 0; i < r; ++i) acc -= am[(b + r) * TP + b + i] * t[i];
+                t[r] = (r >= j) ? acc : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) tm[(b + r) * TP + b + j] = t[r];
+        }
+    } else {
+        for (int idx = tid - 128; idx < C * C; idx += 128) {
+            const int r = idx >> 6, j = idx & 63;
+            if ((j >> 4) > (r >> 4)) tm[r * TP + j] = 0.f;
         }
     }
     __syncthreads();
-    for (int R = 1; R < 4; ++R) {
-        for (int idx = tid; idx < R * 256; idx += THREADS) {
-            const int I = idx >> 8, r = (idx >> 4) & 15, j = idx & 15;
-            float acc = 0.f;
-            for (int J = I; J < R; ++J)
-                for (int m = 0; m < 16; ++m)
-                    acc += am[(R * 16 + r) * TP + J * 16 + m] * tm[(J * 16 + m) * TP + I * 16 + j];
-            y[idx] = acc;
+    {   // 16 -> 32: pairs (0,1) and (2,3); thread -> (pair, row r, columns j, j+8)
+        const int p = tid >> 7, r = (tid >> 3) & 15, j = tid & 7;
+        const int b0 = 32 * p, b1 = b0 + 16;
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float a = am[(b1 + r) * TP + b0 + m];
+            y0 += a * tm[(b0 + m) * TP + b0 + j];
+            y1 += a * tm[(b0 + m) * TP + b0 + j + 8];
         }
+        y[p * 256 + r * 16 + j] = y0;
+        y[p * 256 + r * 16 + j + 8] = y1;
         __syncthreads();
-        for (int idx = tid; idx < R * 256; idx += THREADS) {
-            const int I = idx >> 8, r = (idx >> 4) & 15, j = idx & 15;
-            float acc = 0.f;
-            for (int m = 0; m <= r; ++m) acc += tm[(R * 16 + r) * TP + R * 16 + m] * y[(I << 8) + m * 16 + j];
-            tm[(R * 16 + r) * TP + I * 16 + j] = -acc;
+        float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float tt = tm[(b1 + r) * TP + b1 + m];  // zero above the diagonal
+            t0 += tt * y[p * 256 + m * 16 + j];
+            t1 += tt * y[p * 256 + m * 16 + j + 8];
         }
-        __syncthreads();
+        tm[(b1 + r) * TP + b0 + j] = -t0;
+        tm[(b1 + r) * TP + b0 + j + 8] = -t1;
     }
+    __syncthreads();
+    {   // 32 -> 64: thread -> (row r of the bottom half, columns j, j+8, j+16, j+24)
+        const int r = tid >> 3, j = tid & 7;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+            const float a = am[(32 + r) * TP + m];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] += a * tm[m * TP + j + 8 * q];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) y[r * 32 + j + 8 * q] = acc[q];
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = 0.f;
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+            const float tt = tm[(32 + r) * TP + 32 + m];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] += tt * y[m * 32 + j + 8 * q];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tm[(32 + r) * TP + j + 8 * q] = -acc[q];
+    }
+    __syncthreads();
 }
 
 template <typename TO>
-__device__ __forceinline__ void store_row32(TO* dst, const float (&v)[32]);
+__device__ __forceinline__ void store_row16(TO* dst, const float (&v)[16]);
 template <>
-__device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[32]) {
+__device__ __forceinline__ void store_row16<float>(float* dst, const float (&v)[16]) {
     float4* d = reinterpret_cast<float4*>(dst);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 template <>
-__device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[32]) {
+__device__ __forceinline__ void store_row16<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[16]) {
     uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
         __nv_bfloat162 p0 = __floats2bfloat162_rn(v[8 * i], v[8 * i + 1]);
         __nv_bfloat162 p1 = __floats2bfloat162_rn(v[8 * i + 2], v[8 * i + 3]);
         __nv_bfloat162 p2 = __floats2bfloat162_rn(v[8 * i + 4], v[8 * i + 5]);
@@ -156,21 +217,29 @@ __device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, c
     }
 }
 
-template <typename TG, typename TO>
+template <typename TG>
 __global__ void __launch_bounds__(THREADS, 1)
-chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                const __nv_bfloat16* __restrict__ v, const TG* __restrict__ log_alpha,
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
                 const TG* __restrict__ beta, const float* initial_state, const int32_t* __restrict__ cu_seqlens,
-                int64_t T_total, int N, int H, TO* __restrict__ o, float* final_state, unsigned int* flags) {
+                int64_t T_total, int N, int H, void* __restrict__ o_ptr, int o_is_f32, float* final_state,
+                unsigned int* flags) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
     float* s_beta = tile(sm, OFF_BETA);
+    float* x_part = tile(sm, OFF_XCH);
+    float* x_gm = x_part + 128;
+    float* x_gc = x_part + 256;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* tbar = reinterpret_cast<uint64_t*>(sm + OFF_TBAR);
     uint32_t* slot = reinterpret_cast<uint32_t*>(sm + OFF_SLOT);
     const uint32_t sbase = smem_u32(sm);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3;   // tensor-memory lane quadrant of this warp
+    const int h2 = tid >> 7;   // half: rows 32*h2.. in the elementwise stage, columns 16*h2.. elsewhere
+    const int c = tid & 127;   // key channel / state row
     constexpr int NSLICES = DV / DVS;
     const int64_t blk = blockIdx.x;
     const int slice = static_cast<int>(blk % NSLICES);
@@ -191,111 +260,152 @@ chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         t0 = static_cast<int64_t>(n) * L;
         t1 = t0 + L;
     }
+    constexpr uint32_t kStageBytes = 2 * C * DK * 2 + C * DK * sizeof(TG) + C * DVS * 2;
 
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(tbar, 1);
         fence_mbar_init();
+        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_la); tma_prefetch_desc(&tm_v);
+        if (t0 < t1) {
+            mbar_arrive_expect_tx(tbar, kStageBytes);
+            tma_load_3d(sm + OFF_SK, &tm_k, 0, h, static_cast<int>(t0), tbar);
+            tma_load_3d(sm + OFF_SQ, &tm_q, 0, h, static_cast<int>(t0), tbar);
+            tma_load_3d(sm + OFF_SLA, &tm_la, 0, h, static_cast<int>(t0), tbar);
+            tma_load_3d(sm + OFF_SV, &tm_v, col0, h, static_cast<int>(t0), tbar);
+        }
     }
     if (warp == 0) tmem_alloc(slot, TM_COLS);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *slot;
-    const uint32_t tq = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // this warp's lane quadrant
-    uint32_t phase = 0;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(q4 * 32) << 16);  // this warp's lane quadrant
+    uint32_t phase = 0, tphase = 0;
 
-    const int64_t qk_row = static_cast<int64_t>(H) * DK, v_row = static_cast<int64_t>(H) * DV;
+    const int64_t v_row = static_cast<int64_t>(H) * DV;
     const int64_t state_off = (static_cast<int64_t>(n) * H + h) * DK * DV;
-    const int c = tid;               // key channel / state row owned by this thread
-    const int orow = warp * 16 + lane;  // chunk row owned in the M=64 accumulator layout (lane < 16)
+    const int orow = q4 * 16 + lane;  // chunk row owned in the M=64 accumulator layout (lane < 16)
+    const int scol = col0 + 16 * h2;  // first of the 16 state / output columns this thread owns
 
-    float S[DVS];
+    float S[16];
     if (initial_state) {
-        const float4* src = reinterpret_cast<const float4*>(initial_state + state_off + static_cast<int64_t>(c) * DV + col0);
+        const float4* src = reinterpret_cast<const float4*>(initial_state + state_off + static_cast<int64_t>(c) * DV + scol);
 #pragma unroll
-        for (int i = 0; i < DVS / 4; ++i) {
+        for (int i = 0; i < 4; ++i) {
             const float4 x = src[i];
             S[4 * i] = x.x; S[4 * i + 1] = x.y; S[4 * i + 2] = x.z; S[4 * i + 3] = x.w;
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < DVS; ++j) S[j] = 0.f;
+        for (int j = 0; j < 16; ++j) S[j] = 0.f;
     }
+    float beta_next = 0.f;
+    if (tid < C && t0 + tid < t1) beta_next = to_f32(beta[(t0 + tid) * H + h]);
 
     bool timed_out = false;
+    bool tma_pending = t0 < t1;  // a staging load is in flight and not yet waited for
     for (int64_t c0 = t0; c0 < t1; c0 += C) {
         const int len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
-        if (tid < C) s_beta[tid] = tid < len ? to_f32(beta[(c0 + tid) * H + h]) : 0.f;
+        if (tid < C) s_beta[tid] = beta_next;
+        timed_out = !mbar_wait(tbar, tphase, kWaitPolls);
+        if (__syncthreads_or(timed_out)) break;
+        tphase ^= 1;
+        tma_pending = false;
 
-        // ---- elementwise stage: cumulative log-decay and the anchored operands (thread = channel c)
-        float g[C];
+        // ---- elementwise stage (thread: channel c, rows 32*h2 .. 32*h2+31)
+        const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK);
+        const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ);
+        const TG* sla = reinterpret_cast<const TG*>(sm + OFF_SLA);
+        const int rb = 32 * h2;
+        float g[32];
         {
             float run = 0.f;
-            const TG* la = log_alpha + c0 * qk_row + static_cast<int64_t>(h) * DK + c;
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
-                run += r < len ? to_f32(la[r * qk_row]) : 0.f;
+            for (int r = 0; r < 32; ++r) {
+                run += (rb + r) < len ? to_f32(sla[(rb + r) * DK + c]) : 0.f;
                 g[r] = run;
             }
+            if (h2 == 0) x_part[c] = run;
         }
-        const float gm = g[32], gC = g[C - 1];
-        if (g[0] - gm > kAnchorLimit || gm - gC > kAnchorLimit || gm < -kAnchorLimit)
-            raise_flag(flags, KDA_DEVFLAG_DECAY_RANGE);
+        __syncthreads();
+        if (h2 == 1) {
+            const float off = x_part[c];
+#pragma unroll
+            for (int r = 0; r < 32; ++r) g[r] += off;
+            x_gm[c] = g[0];
+            x_gc[c] = g[31];
+            const float g0 = len > 0 ? to_f32(sla[c]) : 0.f;
+            if (g0 - g[0] > kAnchorLimit || g[0] - g[31] > kAnchorLimit || g[0] < -kAnchorLimit)
+                raise_flag(flags, KDA_DEVFLAG_DECAY_RANGE);
+        }
+        __syncthreads();
+        const float gm = x_gm[c], gC = x_gc[c];
         const float em = expf(gm), ec = expf(gC - gm), gam = expf(gC);
-        {
-            const __nv_bfloat16* kp = k + c0 * qk_row + static_cast<int64_t>(h) * DK + c;
-            const __nv_bfloat16* qp = q + c0 * qk_row + static_cast<int64_t>(h) * DK + c;
+        // rows rb .. rb+31 of channel c -> row c of [K+ | Q+]^T (M-blocks h2 and 2+h2), of (K-)^T
+        // MN-major (N-block h2) and of (K-)^T K-major (K-block h2), four rows per 16-byte store
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
-                const float kv = r < len ? __bfloat162float(kp[r * qk_row]) : 0.f;
-                const float qv = r < len ? __bfloat162float(qp[r * qk_row]) : 0.f;
-                const float e = expf(g[r] - gm), ie = expf(gm - g[r]);
-                const float km = to_tf32(kv * ie);
-                st_sw(sm, OFF_KQ, r, c, 128, to_tf32(kv * e));
-                st_sw(sm, OFF_KQ, C + r, c, 128, to_tf32(qv * e));
-                st_sw(sm, OFF_KM, r, c, 64, km);
-                st_mn(sm, OFF_KMM, r, c, 64, km);
+        for (int r4 = 0; r4 < 32; r4 += 4) {
+            float kp[4], qp[4], km[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = rb + r4 + u;
+                const bool live = r < len;
+                const float kv = live ? __bfloat162float(sk[r * DK + c]) : 0.f;
+                const float qv = live ? __bfloat162float(sq[r * DK + c]) : 0.f;
+                const float e = __expf(g[r4 + u] - gm), ie = __expf(gm - g[r4 + u]);
+                kp[u] = to_tf32(kv * e);
+                qp[u] = to_tf32(qv * e);
+                km[u] = to_tf32(kv * ie);
             }
+            const int m = 32 * h2 + r4;
+            *reinterpret_cast<float4*>(sm + OFF_KQ + sw32b_off(c, m, 128)) = make_float4(kp[0], kp[1], kp[2], kp[3]);
+            *reinterpret_cast<float4*>(sm + OFF_KQ + sw32b_off(c, C + m, 128)) = make_float4(qp[0], qp[1], qp[2], qp[3]);
+            *reinterpret_cast<float4*>(sm + OFF_KM + sw32b_off(c, m, 128)) = make_float4(km[0], km[1], km[2], km[3]);
+            *reinterpret_cast<float4*>(sm + OFF_KMT + sw128_off(c, m, 128)) = make_float4(km[0], km[1], km[2], km[3]);
         }
-        {   // S' = Diag(e^{g_m}) S0, K-row c
-            float sp[DVS];
+        {   // S' = Diag(e^{g_m}) S0: K-row c, columns 16*h2 .. 16*h2+15 of the slice
+            float sp[16];
 #pragma unroll
-            for (int j = 0; j < DVS; ++j) sp[j] = em * S[j];
-#pragma unroll
-            for (int j = 0; j < DVS; j += 8) st_mn8(sm, OFF_S, c, j, 128, sp + j);
+            for (int j = 0; j < 16; ++j) sp[j] = em * S[j];
+            st_mn8(sm, OFF_S, c, 16 * h2, 128, sp);
+            st_mn8(sm, OFF_S, c, 16 * h2 + 8, 128, sp + 8);
         }
-        {   // V slice: thread -> (row, 16 columns)
-            const int r = tid >> 1, j0 = (tid & 1) * 16;
-            float vv[16];
-            if (r < len) {
-                const uint4* src = reinterpret_cast<const uint4*>(v + (c0 + r) * v_row + static_cast<int64_t>(h) * DV + col0 + j0);
-                const uint4 a = src[0], b = src[1];
-                const __nv_bfloat16* pa = reinterpret_cast<const __nv_bfloat16*>(&a);
-                const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(&b);
+        {   // V slice: thread -> (row, 8 columns)
+            const int r = tid >> 2, j0 = (tid & 3) * 8;
+            float vv[8];
+            const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SV) + r * DVS + j0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) { vv[i] = __bfloat162float(pa[i]); vv[8 + i] = __bfloat162float(pb[i]); }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) vv[i] = 0.f;
-            }
-            st_mn8(sm, OFF_V, r, j0, 64, vv);
-            st_mn8(sm, OFF_V, r, j0 + 8, 64, vv + 8);
+            for (int i = 0; i < 8; ++i) vv[i] = r < len ? __bfloat162float(sv[i]) : 0.f;
+            st_mn8(sm, OFF_VD, r, j0, 64, vv);
         }
         fence_async_smem();
         tc_fence_before_sync();
         __syncthreads();
 
+        // ---- prefetch the next chunk's raw tiles (the staging buffer is free now) and its beta
+        const int64_t c1 = c0 + C;
+        if (tid == 0 && c1 < t1) {
+            mbar_arrive_expect_tx(tbar, kStageBytes);
+            tma_load_3d(sm + OFF_SK, &tm_k, 0, h, static_cast<int>(c1), tbar);
+            tma_load_3d(sm + OFF_SQ, &tm_q, 0, h, static_cast<int>(c1), tbar);
+            tma_load_3d(sm + OFF_SLA, &tm_la, 0, h, static_cast<int>(c1), tbar);
+            tma_load_3d(sm + OFF_SV, &tm_v, col0, h, static_cast<int>(c1), tbar);
+        }
+        tma_pending = c1 < t1;
+        if (tid < C) beta_next = (c1 + tid < t1) ? to_f32(beta[(c1 + tid) * H + h]) : 0.f;
+
         // ---- MMA batch 1: [A_raw; P] = [K+; Q+] (K-)^T,  Z = K+ S',  O = Q+ S'
         if (tid == 0) {
             tc_fence_after_sync();
-            const uint32_t id1 = idesc_tf32(128, 64, false, false);
-            const uint32_t idz = idesc_tf32(64, DVS, false, true);
+            const uint32_t id1 = idesc_tf32(128, 64, true, true);
+            const uint32_t idz = idesc_tf32(64, DVS, true, true);
 #pragma unroll
             for (int kk = 0; kk < DK / 8; ++kk) {
-                const uint32_t kofs = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                const uint64_t akq = sw128_desc(sbase + OFF_KQ + kofs, 16, 1024);
-                const uint64_t aq = sw128_desc(sbase + OFF_KQ + kofs + C * 128, 16, 1024);
-                const uint64_t bkm = sw128_desc(sbase + OFF_KM + (kk >> 2) * 64 * 128 + (kk & 3) * 32, 16, 1024);
+                // MN-major tiles: K-step of 8 channels = 8 rows of 128 bytes; 32-column blocks 16 KB apart
+                const uint64_t akq = sw128b32_desc(sbase + OFF_KQ + kk * 1024, 128 * 128, 512);
+                const uint64_t aq = sw128b32_desc(sbase + OFF_KQ + 2 * 128 * 128 + kk * 1024, 128 * 128, 512);
+                const uint64_t bkm = sw128b32_desc(sbase + OFF_KM + kk * 1024, 128 * 128, 512);
                 const uint64_t bs = sw128b32_desc(sbase + OFF_S + kk * 1024, 128 * 128, 512);
                 mma_tf32(tmem + TM_AP, akq, bkm, id1, kk > 0);
                 mma_tf32(tmem + TM_Z, akq, bs, idz, kk > 0);
@@ -308,32 +418,31 @@ chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         if (__syncthreads_or(timed_out)) break;
         tc_fence_after_sync();
         {   // rows 0..63 -> A (fp32, beta-scaled, strictly lower); rows 64..127 -> P (tf32, lower)
-            float* am = tile(sm, OFF_A);
-            const int r = tid & 63;
-            const float br = s_beta[r];
+            float x[32];
+            tmem_ld32(tq + TM_AP + h2 * 32, x);  // M=128: row 32*q4 + lane, columns 32*h2..
+            const int row = q4 * 32 + lane;
+            if (row < C) {
+                float* am = tile(sm, OFF_A);
+                const float br = s_beta[row];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float x[32];
-                tmem_ld32(tq + TM_AP + half * 32, x);
-                if (tid < C) {
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int i = h2 * 32 + jj;
+                    am[row * TP + i] = i < row ? br * x[jj] : 0.f;
+                }
+            } else {
+                const int r = row - C;
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int i = half * 32 + jj;
-                        am[r * TP + i] = i < r ? br * x[jj] : 0.f;
-                    }
-                } else {
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int i = half * 32 + jj;
-                        st_sw(sm, OFF_P, r, i, 64, i <= r ? to_tf32(x[jj]) : 0.f);
-                    }
+                for (int jj = 0; jj < 32; jj += 4) {
+                    const int i = h2 * 32 + jj;
+                    st_sw4(sm, OFF_P, r, i, 64, i <= r ? x[jj] : 0.f, i + 1 <= r ? x[jj + 1] : 0.f,
+                           i + 2 <= r ? x[jj + 2] : 0.f, i + 3 <= r ? x[jj + 3] : 0.f);
                 }
             }
-            float z[32];
-            tmem_ld32(tq + TM_Z, z);  // M=64 layout: row orow in lanes 0..15
+            float z[16];
+            tmem_ld16(tq + TM_Z + h2 * 16, z);  // M=64: row orow in lanes 0..15
             if (lane < 16) {
-#pragma unroll
-                for (int j = 0; j < DVS; j += 8) st_mn8(sm, OFF_Z, orow, j, 64, z + j);
+                st_mn8(sm, OFF_Z, orow, 16 * h2, 64, z);
+                st_mn8(sm, OFF_Z, orow, 16 * h2 + 8, 64, z + 8);
             }
         }
         tc_fence_before_sync();
@@ -342,11 +451,12 @@ chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         // ---- T = (I + A)^{-1}, then T' = T Diag(beta) as an MMA operand
         unit_lower_inverse(tile(sm, OFF_A), tile(sm, OFF_TF), tile(sm, OFF_Y));
         {
-            const float* tf = tile(sm, OFF_TF);
-            for (int idx = tid; idx < C * C; idx += THREADS) {
-                const int r = idx >> 6, i = idx & 63;
-                st_sw(sm, OFF_T, r, i, 64, to_tf32(tf[r * TP + i] * s_beta[i]));
-            }
+            const float* tf = tile(sm, OFF_TF) + (tid >> 2) * TP;
+            const int r = tid >> 2, i0 = (tid & 3) * 16;
+#pragma unroll
+            for (int i = i0; i < i0 + 16; i += 4)
+                st_sw4(sm, OFF_T, r, i, 64, tf[i] * s_beta[i], tf[i + 1] * s_beta[i + 1], tf[i + 2] * s_beta[i + 2],
+                       tf[i + 3] * s_beta[i + 3]);
         }
         fence_async_smem();
         tc_fence_before_sync();
@@ -359,7 +469,7 @@ chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk) {
                 const uint64_t at = sw128_desc(sbase + OFF_T + (kk >> 2) * 64 * 128 + (kk & 3) * 32, 16, 1024);
-                const uint64_t bv = sw128b32_desc(sbase + OFF_V + kk * 1024, 64 * 128, 512);
+                const uint64_t bv = sw128b32_desc(sbase + OFF_VD + kk * 1024, 64 * 128, 512);
                 const uint64_t bz = sw128b32_desc(sbase + OFF_Z + kk * 1024, 64 * 128, 512);
                 mma_tf32(tmem + TM_U, at, bv, id, kk > 0);
                 mma_tf32(tmem + TM_X, at, bz, id, kk > 0);
@@ -370,15 +480,15 @@ chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         phase ^= 1;
         if (__syncthreads_or(timed_out)) break;
         tc_fence_after_sync();
-        {   // Delta = U - X  (rows in the M=64 layout)
-            float u[32], x[32];
-            tmem_ld32(tq + TM_U, u);
-            tmem_ld32(tq + TM_X, x);
+        {   // Delta = U - X  (rows in the M=64 layout, columns 16*h2..)
+            float u[16], x[16];
+            tmem_ld16(tq + TM_U + h2 * 16, u);
+            tmem_ld16(tq + TM_X + h2 * 16, x);
             if (lane < 16) {
 #pragma unroll
-                for (int j = 0; j < DVS; ++j) u[j] -= x[j];
-#pragma unroll
-                for (int j = 0; j < DVS; j += 8) st_mn8(sm, OFF_D, orow, j, 64, u + j);
+                for (int j = 0; j < 16; ++j) u[j] -= x[j];
+                st_mn8(sm, OFF_VD, orow, 16 * h2, 64, u);
+                st_mn8(sm, OFF_VD, orow, 16 * h2 + 8, 64, u + 8);
             }
         }
         fence_async_smem();
@@ -388,13 +498,13 @@ chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         // ---- MMA batch 3: Y = (K-)^T Delta (A MN-major),  O += P Delta
         if (tid == 0) {
             tc_fence_after_sync();
-            const uint32_t idy = idesc_tf32(128, DVS, true, true);
+            const uint32_t idy = idesc_tf32(128, DVS, false, true);
             const uint32_t ido = idesc_tf32(64, DVS, false, true);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk) {
-                const uint64_t ak = sw128b32_desc(sbase + OFF_KMM + kk * 1024, 64 * 128, 512);
+                const uint64_t ak = sw128_desc(sbase + OFF_KMT + (kk >> 2) * 128 * 128 + (kk & 3) * 32, 16, 1024);
                 const uint64_t ap = sw128_desc(sbase + OFF_P + (kk >> 2) * 64 * 128 + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = sw128b32_desc(sbase + OFF_D + kk * 1024, 64 * 128, 512);
+                const uint64_t bd = sw128b32_desc(sbase + OFF_VD + kk * 1024, 64 * 128, 512);
                 mma_tf32(tmem + TM_Y, ak, bd, idy, kk > 0);
                 mma_tf32(tmem + TM_O, ap, bd, ido, 1);
             }
@@ -405,56 +515,92 @@ chunk_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         if (__syncthreads_or(timed_out)) break;
         tc_fence_after_sync();
         {
-            float y[32];
-            tmem_ld32(tq + TM_Y, y);  // M=128: lane = state row c
+            float y[16];
+            tmem_ld16(tq + TM_Y + h2 * 16, y);  // M=128: lane = state row c
 #pragma unroll
-            for (int j = 0; j < DVS; ++j) S[j] = gam * S[j] + ec * y[j];
-            float ov[32];
-            tmem_ld32(tq + TM_O, ov);
-            if (lane < 16 && orow < len)
-                store_row32<TO>(o + (c0 + orow) * v_row + static_cast<int64_t>(h) * DV + col0, ov);
+            for (int j = 0; j < 16; ++j) S[j] = gam * S[j] + ec * y[j];
+            float ov[16];
+            tmem_ld16(tq + TM_O + h2 * 16, ov);
+            if (lane < 16 && orow < len) {
+                const int64_t off = (c0 + orow) * v_row + static_cast<int64_t>(h) * DV + scol;
+                if (o_is_f32) store_row16<float>(static_cast<float*>(o_ptr) + off, ov);
+                else store_row16<__nv_bfloat16>(static_cast<__nv_bfloat16*>(o_ptr) + off, ov);
+            }
         }
         tc_fence_before_sync();
         __syncthreads();
     }
 
     if (timed_out) {
+        // leave no copy into this CTA's shared memory behind: wait (bounded) for the staging load
+        if (tma_pending) mbar_wait(tbar, tphase, kWaitPolls);
         if (tid == 0) raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
     } else if (final_state) {
-        float4* dst = reinterpret_cast<float4*>(final_state + state_off + static_cast<int64_t>(c) * DV + col0);
+        float4* dst = reinterpret_cast<float4*>(final_state + state_off + static_cast<int64_t>(c) * DV + scol);
 #pragma unroll
-        for (int i = 0; i < DVS / 4; ++i) dst[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) dst[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
     }
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
-template <typename TG, typename TO>
+// ---- host side: TMA descriptors for the [T, H, d] inputs (3-D: d innermost, then heads, then tokens)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t box0, uint32_t box2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+    const cuuint32_t box[3] = {box0, 1, box2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename TG>
 cudaError_t launch_typed(const ChunkArgs& a) {
-    auto kern = chunk_tc_kernel<TG, TO>;
+    CUtensorMap mq, mk, mla, mv;
+    const uint64_t T = static_cast<uint64_t>(a.T_total), H = static_cast<uint64_t>(a.H);
+    const CUtensorMapDataType gdt = sizeof(TG) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!encode_3d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, H, T, DK, C) ||
+        !encode_3d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, H, T, DK, C) ||
+        !encode_3d(&mla, a.log_alpha, gdt, sizeof(TG), DK, H, T, DK, C) ||
+        !encode_3d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, H, T, DVS, C))
+        return cudaErrorInvalidValue;
+    auto kern = chunk_tc_kernel<TG>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int64_t blocks = static_cast<int64_t>(a.N) * a.H * (DV / DVS);
     kern<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
-        static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-        static_cast<const __nv_bfloat16*>(a.v), static_cast<const TG*>(a.log_alpha),
-        static_cast<const TG*>(a.beta), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H,
-        static_cast<TO*>(a.o), a.final_state, a.flags);
+        mq, mk, mla, mv, static_cast<const TG*>(a.beta), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
+        a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 bool chunk_tc_supported(const ChunkArgs& a) {
-    return a.dtype_qkv == KDA_BF16 && a.dk == DK && a.dv == DV;
+    // T_total = 0 has no tile to describe; the CUDA-core path passes the states through.
+    return a.dtype_qkv == KDA_BF16 && a.dk == DK && a.dv == DV && a.T_total > 0 && a.T_total < (int64_t(1) << 31);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs& a) {
-    if (a.dtype_gate == KDA_FP32)
-        return a.dtype_o == KDA_FP32 ? launch_typed<float, float>(a) : launch_typed<float, __nv_bfloat16>(a);
-    return a.dtype_o == KDA_FP32 ? launch_typed<__nv_bfloat16, float>(a)
-                                 : launch_typed<__nv_bfloat16, __nv_bfloat16>(a);
+    return a.dtype_gate == KDA_FP32 ? launch_typed<float>(a) : launch_typed<__nv_bfloat16>(a);
 }
 
 size_t chunk_tc_workspace_size(int64_t, int, int, int, int) { return 0; }
