@@ -95,12 +95,6 @@ constexpr uint32_t TM_COLS = 128;
 __device__ __forceinline__ float* tile(unsigned char* base, uint32_t off) {
     return reinterpret_cast<float*>(base + off);
 }
-__device__ __forceinline__ void st_sw(unsigned char* base, uint32_t off, int row, int col, int rows, float x) {
-    *reinterpret_cast<float*>(base + off + sw128_off(row, col, rows)) = x;
-}
-__device__ __forceinline__ void st_mn(unsigned char* base, uint32_t off, int k_row, int col, int rows, float x) {
-    *reinterpret_cast<float*>(base + off + sw32b_off(k_row, col, rows)) = x;
-}
 // Eight consecutive M/N elements (col multiple of 8) of one K-row of an MN-major tile, rounded to tf32.
 __device__ __forceinline__ void st_mn8(unsigned char* base, uint32_t off, int k_row, int col, int rows,
                                        const float* x) {
@@ -303,6 +297,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float beta_next = 0.f;
     if (tid < C && t0 + tid < t1) beta_next = to_f32(beta[(t0 + tid) * H + h]);
 
+    // Matrix descriptors at K-step 0; K-step kk adds its byte offset >> 4 to the start-address field.
+    const uint64_t d_kq = sw128b32_desc(sbase + OFF_KQ, 128 * 128, 512);      // [K+|Q+]^T, MN-major
+    const uint64_t d_km = sw128b32_desc(sbase + OFF_KM, 128 * 128, 512);      // (K-)^T, MN-major
+    const uint64_t d_s = sw128b32_desc(sbase + OFF_S, 128 * 128, 512);        // S', MN-major
+    const uint64_t d_t = sw128_desc(sbase + OFF_T, 16, 1024);                 // T', K-major
+    const uint64_t d_v = sw128b32_desc(sbase + OFF_VD, 64 * 128, 512);        // V / Delta, MN-major
+    const uint64_t d_z = sw128b32_desc(sbase + OFF_Z, 64 * 128, 512);         // Z, MN-major
+    const uint64_t d_kmt = sw128_desc(sbase + OFF_KMT, 16, 1024);             // (K-)^T, K-major
+    const uint64_t d_p = sw128_desc(sbase + OFF_P, 16, 1024);                 // P, K-major
+    constexpr uint64_t kQplus = (2 * 128 * 128) >> 4;                          // Q+ M-blocks
     bool timed_out = false;
     bool tma_pending = t0 < t1;  // a staging load is in flight and not yet waited for
     for (int64_t c0 = t0; c0 < t1; c0 += C) {
@@ -402,11 +406,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t idz = idesc_tf32(64, DVS, true, true);
 #pragma unroll
             for (int kk = 0; kk < DK / 8; ++kk) {
-                // MN-major tiles: K-step of 8 channels = 8 rows of 128 bytes; 32-column blocks 16 KB apart
-                const uint64_t akq = sw128b32_desc(sbase + OFF_KQ + kk * 1024, 128 * 128, 512);
-                const uint64_t aq = sw128b32_desc(sbase + OFF_KQ + 2 * 128 * 128 + kk * 1024, 128 * 128, 512);
-                const uint64_t bkm = sw128b32_desc(sbase + OFF_KM + kk * 1024, 128 * 128, 512);
-                const uint64_t bs = sw128b32_desc(sbase + OFF_S + kk * 1024, 128 * 128, 512);
+                // MN-major tiles: K-step of 8 channels = 8 rows of 128 bytes (1024 >> 4 = 64)
+                const uint64_t step = static_cast<uint64_t>(kk) * 64;
+                const uint64_t akq = d_kq + step, aq = d_kq + kQplus + step;
+                const uint64_t bkm = d_km + step, bs = d_s + step;
                 mma_tf32(tmem + TM_AP, akq, bkm, id1, kk > 0);
                 mma_tf32(tmem + TM_Z, akq, bs, idz, kk > 0);
                 mma_tf32(tmem + TM_O, aq, bs, idz, kk > 0);
@@ -468,9 +471,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t id = idesc_tf32(64, DVS, false, true);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk) {
-                const uint64_t at = sw128_desc(sbase + OFF_T + (kk >> 2) * 64 * 128 + (kk & 3) * 32, 16, 1024);
-                const uint64_t bv = sw128b32_desc(sbase + OFF_VD + kk * 1024, 64 * 128, 512);
-                const uint64_t bz = sw128b32_desc(sbase + OFF_Z + kk * 1024, 64 * 128, 512);
+                const uint64_t at = d_t + (((kk >> 2) * 64 * 128 + (kk & 3) * 32) >> 4);
+                const uint64_t bv = d_v + static_cast<uint64_t>(kk) * 64;
+                const uint64_t bz = d_z + static_cast<uint64_t>(kk) * 64;
                 mma_tf32(tmem + TM_U, at, bv, id, kk > 0);
                 mma_tf32(tmem + TM_X, at, bz, id, kk > 0);
             }
@@ -502,9 +505,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t ido = idesc_tf32(64, DVS, false, true);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk) {
-                const uint64_t ak = sw128_desc(sbase + OFF_KMT + (kk >> 2) * 128 * 128 + (kk & 3) * 32, 16, 1024);
-                const uint64_t ap = sw128_desc(sbase + OFF_P + (kk >> 2) * 64 * 128 + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = sw128b32_desc(sbase + OFF_VD + kk * 1024, 64 * 128, 512);
+                const uint64_t ak = d_kmt + (((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4);
+                const uint64_t ap = d_p + (((kk >> 2) * 64 * 128 + (kk & 3) * 32) >> 4);
+                const uint64_t bd = d_v + static_cast<uint64_t>(kk) * 64;
                 mma_tf32(tmem + TM_Y, ak, bd, idy, kk > 0);
                 mma_tf32(tmem + TM_O, ap, bd, ido, 1);
             }

@@ -154,11 +154,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// fp32 -> tf32 (round to nearest, ties away), kept in a 32-bit container
+// fp32 -> tf32 (10 mantissa bits), round to nearest with ties away from zero, kept in a 32-bit
+// container.  Done on the integer pipe: add half an ulp of the tf32 grid (bit 12) to the magnitude
+// bits and clear the 13 bits tf32 drops; a carry out of the mantissa correctly bumps the exponent.
 __device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
 // Byte offset of element (row, col) of a fp32 tile stored in 128-byte-swizzled column blocks of 32
