@@ -37,7 +37,7 @@ def _rand_inputs(rng, T, H, dk, dv, N_state=1):
     return q, k, v, la, beta, s0
 
 
-def test_hand_worked_example():
+def test_hand_worked_example(fwd=oracle.forward):
     with open(os.path.join(GOLDEN, "kda_hand_example.json")) as f:
         ex = json.load(f)
     q = np.array(ex["q"])[:, None, :]
@@ -46,7 +46,7 @@ def test_hand_worked_example():
     la = np.log(np.array(ex["alpha"]))[:, None, :]
     beta = np.array(ex["beta"])[:, None]
     s0 = np.array(ex["S0"], dtype=np.float64)[None, None]
-    o, sf = oracle.forward(q, k, v, la, beta, s0)
+    o, sf = fwd(q, k, v, la, beta, s0)
     np.testing.assert_allclose(o[:, 0, :], np.array(ex["o"]), rtol=0, atol=1e-14)
     np.testing.assert_allclose(sf[0, 0], np.array(ex["S_final"]), rtol=0, atol=1e-14)
 
@@ -103,25 +103,25 @@ def _gdn_textbook(q, k, v, alpha, beta, s0):
     return np.array(out), S
 
 
-def test_scalar_alpha_reduces_to_gated_deltanet():
+def test_scalar_alpha_reduces_to_gated_deltanet(fwd=oracle.forward):
     rng = np.random.default_rng(3)
     T, H, dk, dv = 24, 2, 5, 4
     q, k, v, _, beta, s0 = _rand_inputs(rng, T, H, dk, dv)
     a_scalar = -np.exp(rng.uniform(-3.0, -0.7, (T, H)))  # short T keeps 1/gamma moderate
     la = np.repeat(a_scalar[:, :, None], dk, axis=2)
-    o, sf = oracle.forward(q, k, v, la, beta, s0)
+    o, sf = fwd(q, k, v, la, beta, s0)
     for h in range(H):
         o_ref, s_ref = _gdn_textbook(q[:, h], k[:, h], v[:, h], np.exp(a_scalar[:, h]), beta[:, h], s0[0, h])
         np.testing.assert_allclose(o[:, h], o_ref, rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(sf[0, h], s_ref, rtol=1e-12, atol=1e-12)
     # rescaling identity: GDN(v) = gamma_t * DeltaNet(v / gamma_t), gamma_t = prod_{j<=t} alpha_j
     gamma = np.exp(np.cumsum(a_scalar, axis=0))  # [T, H]
-    o_dn, sf_dn = oracle.forward(q, k, v / gamma[:, :, None], np.zeros_like(la), beta, s0)
+    o_dn, sf_dn = fwd(q, k, v / gamma[:, :, None], np.zeros_like(la), beta, s0)
     np.testing.assert_allclose(o, gamma[:, :, None] * o_dn, rtol=1e-9, atol=1e-12)
     np.testing.assert_allclose(sf[0], gamma[-1][:, None, None] * sf_dn[0], rtol=1e-9, atol=1e-12)
 
 
-def test_write_read_invariant():
+def test_write_read_invariant(fwd=oracle.forward):
     """With ||k_t|| = 1 and beta_t = 1 the state returns v_t for key k_t right after the write."""
     rng = np.random.default_rng(4)
     T, H, dk, dv = 40, 2, 8, 5
@@ -129,7 +129,7 @@ def test_write_read_invariant():
     beta = np.ones((T, H))
     S = s0
     for t in range(T):
-        _, S = oracle.forward(q[t:t + 1], k[t:t + 1], v[t:t + 1], la[t:t + 1], beta[t:t + 1], S)
+        _, S = fwd(q[t:t + 1], k[t:t + 1], v[t:t + 1], la[t:t + 1], beta[t:t + 1], S)
         for h in range(H):
             read = S[0, h].T @ k[t, h]
             assert np.linalg.norm(read - v[t, h]) <= 1e-12 * np.linalg.norm(v[t, h])
@@ -140,7 +140,7 @@ def _frac_vec(xs):
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
-def test_brute_force_transition_product(seed):
+def test_brute_force_transition_product(seed, fwd=oracle.forward):
     """S_T = (prod_{j=T..1} M_j) S0 + sum_i (prod_{j=T..i+1} M_j) beta_i k_i v_i^T with
     M_j = (I - beta_j k_j k_j^T) Diag(alpha_j), in exact rationals over dyadic inputs."""
     rng = np.random.default_rng(100 + seed)
@@ -184,8 +184,7 @@ def test_brute_force_transition_product(seed):
         o_exact.append([float(sum((S[r][c] * qt[r] for r in range(dk)), Fraction(0))) for c in range(dv)])
     S_exact = np.array([[float(x) for x in row] for row in S])
 
-    o, sf = oracle.forward(q[:, None], k[:, None], v[:, None], np.log(alpha)[:, None], beta[:, None],
-                           s0[None, None])
+    o, sf = fwd(q[:, None], k[:, None], v[:, None], np.log(alpha)[:, None], beta[:, None], s0[None, None])
     # log(alpha) then exp() in the oracle costs a few ulp per factor
     np.testing.assert_allclose(o[:, 0], np.array(o_exact), rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(sf[0, 0], S_exact, rtol=1e-12, atol=1e-13)
