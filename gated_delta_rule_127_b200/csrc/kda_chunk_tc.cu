@@ -13,16 +13,16 @@
 //   S' = Diag(e^{g_m}) S0
 //   [A_raw; P] = [K+; Q+] (K-)^T,  Z = K+ S',  O = Q+ S'       MMA batch 1
 //   A = beta_r A_raw (strictly lower);  P lower with diagonal
-//   T = (I + A)^{-1}                                          forward substitution, CUDA cores, fp32
-//   T' = T Diag(beta)
-//   U = T' V,  X = T' Z                                       MMA batch 2
-//   Delta = U - X
-//   Y = (K-)^T Delta,  O += P Delta                           MMA batch 3
+//   (I + A) Delta = Diag(beta) (V - Z)                        blocked forward substitution, fp32
+//   Y = (K-)^T Delta,  O += P Delta                           MMA batch 2
 //   S_C = Diag(e^{g_C}) S0 + Diag(e^{g_C - g_m}) Y;   o = O
-// This is the usual WY/UT form U = T Diag(beta) V, W = T Diag(beta) (K e^G), Delta = U - W S0,
-// O = (Q e^G) S0 + P Delta, S_C = Diag(e^{g_C}) S0 + (K e^{g_C - G})^T Delta, evaluated with W S0
-// associated as T' (K+ S') (no W tile, fewer flops per dv slice), and with the per-channel factors
-// e^{g_m} and e^{g_C - g_m} moved onto S0 and onto the MMA result so no operand is scaled twice.
+// This is the WY/UT form Delta = U - W S0 with U = T Diag(beta) V, W = T Diag(beta) (K e^G) and
+// T = (I + A)^{-1}: since Z = (K e^G) S0, Delta = T Diag(beta) (V - Z), which the kernel obtains by
+// forward substitution over 16-row blocks -- each diagonal block's inverse (I + A_RR)^{-1} by
+// forward substitution in registers, the blocks below updated with A_R'R Delta_R -- so the full
+// 64 x 64 inverse is never formed.  O = (Q e^G) S0 + P Delta and
+// S_C = Diag(e^{g_C}) S0 + (K e^{g_C - G})^T Delta, with the per-channel factors e^{g_m} and
+// e^{g_C - g_m} moved onto S0 and onto the MMA result so that no operand is scaled twice.
 // The anchor split e^{g_r - g_i} = e^{g_r - g_m} e^{g_m - g_i} keeps every factor that can exceed 1
 // below e^80 while the chunk's log-decay stays within 80 of g_m at both ends ("일반 DPLR보다 줄어든
 // 연산량" on the same page notes that fine-grained decay makes intra-chunk division numerically
@@ -34,10 +34,11 @@
 // about 5e-3.  K-major operands use the 128-byte swizzle; MN-major tf32 operands must use the
 // 128-byte layout with 32-byte atoms.
 //
-// One CTA of 256 threads owns one (sequence, head, 32-column slice of dv) and walks its chunks in
+// One CTA of 512 threads owns one (sequence, head, 32-column slice of dv) and walks its chunks in
 // order.  The raw q, k, log_alpha and v tiles of the next chunk are brought into shared memory by
 // TMA while the current chunk computes.  Thread t owns key channel / state row c = t % 128 and
-// half h2 = t / 128 of that channel's rows in the elementwise stage and of the state row's columns.
+// quarter qr = t / 128: rows 16 qr .. 16 qr + 15 of that channel in the elementwise stage, and
+// columns 8 qr .. 8 qr + 7 of the state row and of the chunk's output rows.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -56,8 +57,8 @@ constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DV = 128;
 constexpr int DVS = 32;
-constexpr int THREADS = 256;
-constexpr int TP = 65;              // padded row stride of the fp32 A and T tiles
+constexpr int THREADS = 512;
+constexpr int TP = 68;              // row stride of the fp32 A and T tiles (16-byte aligned rows)
 constexpr float kAnchorLimit = 80.f;
 constexpr uint32_t kWaitPolls = 1u << 26;
 
@@ -66,30 +67,30 @@ constexpr uint32_t kWaitPolls = 1u << 26;
 // operand tiles of the elementwise stage are stored transposed (row = key channel c), so each
 // thread writes whole rows of its own channel with 16-byte stores.
 constexpr uint32_t OFF_KQ = 0;         // [K+ | Q+]^T  MN-major, K-rows c (128) x M-cols r (128): 64 KB
-constexpr uint32_t OFF_A = 0;          //   after batch 1: A  fp32 [64][65]
-constexpr uint32_t OFF_TF = 16640;     //                  T  fp32 [64][65]
-constexpr uint32_t OFF_T = 33792;      //                  T' K-major 64 x 64 (16 KB)
-constexpr uint32_t OFF_Y = 50176;      //                  1024 floats of block-inverse scratch
+constexpr uint32_t OFF_A = 0;          //   after batch 1: A  fp32 [64][68]
+constexpr uint32_t OFF_TF = 17408;     //                  diagonal-block inverses fp32 [64][68]
+constexpr uint32_t OFF_DL = 34816;     //                  Delta fp32 [64][32]
 constexpr uint32_t OFF_KM = 65536;     // (K-)^T  MN-major, K-rows c (128) x N-cols i (64): 32 KB
 constexpr uint32_t OFF_P = 65536;      //   after batch 1: P  K-major 64 x 64 (16 KB)
-constexpr uint32_t OFF_Z = 81920;      //                  Z  MN-major 64 x 32 (8 KB)
+constexpr uint32_t OFF_D = 81920;      //                  Delta MN-major 64 x 32 (8 KB)
 constexpr uint32_t OFF_KMT = 98304;    // (K-)^T  K-major, rows c (128) x K-cols i (64): 32 KB
 constexpr uint32_t OFF_S = 131072;     // S'  MN-major 128 x 32 (16 KB)
-constexpr uint32_t OFF_VD = 147456;    // V, then Delta: MN-major 64 x 32 (8 KB)
+constexpr uint32_t OFF_R = 147456;     // right-hand side beta (V - Z), fp32 [64][32] (8 KB)
 constexpr uint32_t OFF_SK = 155648;    // TMA staging: k   bf16 [64][128]
 constexpr uint32_t OFF_SQ = 172032;    //              q   bf16 [64][128]
 constexpr uint32_t OFF_SLA = 188416;   //              log_alpha [64][128] (fp32 or bf16)
 constexpr uint32_t OFF_SV = 221184;    //              v   bf16 [64][32]
 constexpr uint32_t OFF_BETA = 225280;  // 64 floats
-constexpr uint32_t OFF_XCH = 225536;   // 3 x 128 floats: half-column sums, g at row 32, g at row 63
-constexpr uint32_t OFF_BAR = 227072;   // mbarrier: MMA completion
-constexpr uint32_t OFF_TBAR = 227080;  // mbarrier: TMA completion
-constexpr uint32_t OFF_SLOT = 227088;  // tensor-memory base address
-constexpr uint32_t SMEM_USED = 227096;
+constexpr uint32_t OFF_XCH = 225536;   // 6 x 128 floats: quarter-column sums, g at row 32, g at row 63
+constexpr uint32_t OFF_BAR = 228608;   // mbarrier: MMA completion
+constexpr uint32_t OFF_TBAR = 228616;  // mbarrier: TMA completion
+constexpr uint32_t OFF_SLOT = 228624;  // tensor-memory base address
+constexpr uint32_t OFF_BAR2 = 228632;  // mbarrier: completion of the second half of MMA batch 1
+constexpr uint32_t SMEM_USED = 228640;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 
-// Tensor-memory columns (fp32).  Batch 2 and 3 reuse the columns batch 1 results were read from.
-constexpr uint32_t TM_AP = 0, TM_Z = 64, TM_O = 96, TM_U = 0, TM_X = 32, TM_Y = 64;
+// Tensor-memory columns (fp32).  Batch 2 writes Y into the columns Z was read from.
+constexpr uint32_t TM_AP = 0, TM_Z = 64, TM_O = 96, TM_Y = 64;
 constexpr uint32_t TM_COLS = 128;
 
 __device__ __forceinline__ float* tile(unsigned char* base, uint32_t off) {
@@ -103,6 +104,12 @@ __device__ __forceinline__ void st_mn8(unsigned char* base, uint32_t off, int k_
     d[1] = make_float4(to_tf32(x[4]), to_tf32(x[5]), to_tf32(x[6]), to_tf32(x[7]));
 }
 
+// Four consecutive M/N elements (col multiple of 4) of one K-row of an MN-major tile, rounded to tf32.
+__device__ __forceinline__ void st_mn4(unsigned char* base, uint32_t off, int k_row, int col, int rows,
+                                       const float* x) {
+    *reinterpret_cast<float4*>(base + off + sw32b_off(k_row, col, rows)) =
+        make_float4(to_tf32(x[0]), to_tf32(x[1]), to_tf32(x[2]), to_tf32(x[3]));
+}
 // Four consecutive elements (col multiple of 4) of one row of a K-major tile, rounded to tf32.
 __device__ __forceinline__ void st_sw4(unsigned char* base, uint32_t off, int row, int col, int rows,
                                        float a, float b, float c, float d) {
@@ -110,105 +117,89 @@ __device__ __forceinline__ void st_sw4(unsigned char* base, uint32_t off, int ro
         make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
 
-// T = (I + A)^{-1} for strictly lower A (64 x 64, fp32, row stride TP), by forward substitution:
-// inside each 16 x 16 diagonal block column by column (registers), then doubling the solved
-// block: for [T11 0; T21 T22] with T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1},
-// T21 = -T22 (A21 T11) -- first for 16 -> 32 (two blocks at once), then 32 -> 64.
-__device__ void unit_lower_inverse(const float* am, float* tm, float* y) {
+// Inverses of the four 16 x 16 diagonal blocks of I + A (A strictly lower, fp32, row stride TP),
+// by forward substitution, one column per lane (registers): t = (I + A_RR)^{-1}, zero above the
+// diagonal.  Warps 0..3 each take one block.
+__device__ __forceinline__ void diag_block_inverses(const float* am, float* tm) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (warp < 4) {
-        if (lane < 16) {
-            const int b = warp * 16, j = lane;
-            float t[16];
+    if (warp < 4 && lane < 16) {
+        const int b = warp * 16, j = lane;
+        float t[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = (r == j) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int i = 0; i < r; ++i) acc -= am[(b + r) * TP + b + i] * t[i];
-                t[r] = (r >= j) ? acc : 0.f;
+            for (int i = 0; i < r; ++i) acc -= am[(b + r) * TP + b + i] * t[i];
+            t[r] = (r >= j) ? acc : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) tm[(b + r) * TP + b + j] = t[r];
+    }
+}
+
+// Solves (I + A) D = R (64 x 32, fp32) by block forward substitution over four 16-row blocks:
+// D_R = (I + A_RR)^{-1} R_R, then R_R' -= A_R'R D_R for every block R' below.  R is overwritten.
+// Thread t handles column j = t % 32 and row t / 32 of every 16-row block: one warp per row, so the
+// rows of A and of the diagonal-block inverses are warp-wide float4 broadcasts, and the update
+// reuses the column of D_R it loads for all the blocks below.  Writes D as the tf32 MN-major
+// operand tile at `off_d`.
+__device__ __forceinline__ void block_forward_solve(const float* am, const float* tm, float* rh, float* dl,
+                                                    unsigned char* sm, uint32_t off_d) {
+    const int tid = threadIdx.x;
+    const int r = tid >> 5, j = tid & 31;  // 16 rows x 32 columns
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+        const int b = 16 * blk;
+        {
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 t = *reinterpret_cast<const float4*>(tm + (b + r) * TP + b + 4 * k);
+                acc += t.x * rh[(b + 4 * k) * DVS + j] + t.y * rh[(b + 4 * k + 1) * DVS + j] +
+                       t.z * rh[(b + 4 * k + 2) * DVS + j] + t.w * rh[(b + 4 * k + 3) * DVS + j];
             }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) tm[(b + r) * TP + b + j] = t[r];
+            dl[(b + r) * DVS + j] = acc;
+            *reinterpret_cast<float*>(sm + off_d + sw32b_off(b + r, j, 64)) = to_tf32(acc);
         }
-    } else {
-        for (int idx = tid - 128; idx < C * C; idx += 128) {
-            const int r = idx >> 6, j = idx & 63;
-            if ((j >> 4) > (r >> 4)) tm[r * TP + j] = 0.f;
-        }
-    }
-    __syncthreads();
-    {   // 16 -> 32: pairs (0,1) and (2,3); thread -> (pair, row r, columns j, j+8)
-        const int p = tid >> 7, r = (tid >> 3) & 15, j = tid & 7;
-        const int b0 = 32 * p, b1 = b0 + 16;
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float a = am[(b1 + r) * TP + b0 + m];
-            y0 += a * tm[(b0 + m) * TP + b0 + j];
-            y1 += a * tm[(b0 + m) * TP + b0 + j + 8];
-        }
-        y[p * 256 + r * 16 + j] = y0;
-        y[p * 256 + r * 16 + j + 8] = y1;
         __syncthreads();
-        float t0 = 0.f, t1 = 0.f;
+        if (blk < 3) {
+            float d[16];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float tt = tm[(b1 + r) * TP + b1 + m];  // zero above the diagonal
-            t0 += tt * y[p * 256 + m * 16 + j];
-            t1 += tt * y[p * 256 + m * 16 + j + 8];
+            for (int m = 0; m < 16; ++m) d[m] = dl[(b + m) * DVS + j];
+#pragma unroll
+            for (int nb = blk + 1; nb < 4; ++nb) {
+                const int row = 16 * nb + r;
+                float acc = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 a = *reinterpret_cast<const float4*>(am + row * TP + b + 4 * k);
+                    acc += a.x * d[4 * k] + a.y * d[4 * k + 1] + a.z * d[4 * k + 2] + a.w * d[4 * k + 3];
+                }
+                rh[row * DVS + j] -= acc;
+            }
+            __syncthreads();
         }
-        tm[(b1 + r) * TP + b0 + j] = -t0;
-        tm[(b1 + r) * TP + b0 + j + 8] = -t1;
     }
-    __syncthreads();
-    {   // 32 -> 64: thread -> (row r of the bottom half, columns j, j+8, j+16, j+24)
-        const int r = tid >> 3, j = tid & 7;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 32; ++m) {
-            const float a = am[(32 + r) * TP + m];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[q] += a * tm[m * TP + j + 8 * q];
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) y[r * 32 + j + 8 * q] = acc[q];
-        __syncthreads();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q] = 0.f;
-#pragma unroll
-        for (int m = 0; m < 32; ++m) {
-            const float tt = tm[(32 + r) * TP + 32 + m];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[q] += tt * y[m * 32 + j + 8 * q];
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tm[(32 + r) * TP + j + 8 * q] = -acc[q];
-    }
-    __syncthreads();
 }
 
 template <typename TO>
-__device__ __forceinline__ void store_row16(TO* dst, const float (&v)[16]);
+__device__ __forceinline__ void store_row8(TO* dst, const float (&v)[8]);
 template <>
-__device__ __forceinline__ void store_row16<float>(float* dst, const float (&v)[16]) {
+__device__ __forceinline__ void store_row8<float>(float* dst, const float (&v)[8]) {
     float4* d = reinterpret_cast<float4*>(dst);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    d[0] = make_float4(v[0], v[1], v[2], v[3]);
+    d[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 template <>
-__device__ __forceinline__ void store_row16<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[16]) {
-    uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        __nv_bfloat162 p0 = __floats2bfloat162_rn(v[8 * i], v[8 * i + 1]);
-        __nv_bfloat162 p1 = __floats2bfloat162_rn(v[8 * i + 2], v[8 * i + 3]);
-        __nv_bfloat162 p2 = __floats2bfloat162_rn(v[8 * i + 4], v[8 * i + 5]);
-        __nv_bfloat162 p3 = __floats2bfloat162_rn(v[8 * i + 6], v[8 * i + 7]);
-        uint4 u;
-        u.x = *reinterpret_cast<uint32_t*>(&p0); u.y = *reinterpret_cast<uint32_t*>(&p1);
-        u.z = *reinterpret_cast<uint32_t*>(&p2); u.w = *reinterpret_cast<uint32_t*>(&p3);
-        d[i] = u;
-    }
+__device__ __forceinline__ void store_row8<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[8]) {
+    __nv_bfloat162 p0 = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 p1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 p2 = __floats2bfloat162_rn(v[4], v[5]);
+    __nv_bfloat162 p3 = __floats2bfloat162_rn(v[6], v[7]);
+    uint4 u;
+    u.x = *reinterpret_cast<uint32_t*>(&p0); u.y = *reinterpret_cast<uint32_t*>(&p1);
+    u.z = *reinterpret_cast<uint32_t*>(&p2); u.w = *reinterpret_cast<uint32_t*>(&p3);
+    *reinterpret_cast<uint4*>(dst) = u;
 }
 
 template <typename TG>
@@ -222,17 +213,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
     float* s_beta = tile(sm, OFF_BETA);
-    float* x_part = tile(sm, OFF_XCH);
-    float* x_gm = x_part + 128;
-    float* x_gc = x_part + 256;
+    float* x_part = tile(sm, OFF_XCH);      // [4][128] quarter-column sums of log_alpha
+    float* x_gm = x_part + 512;
+    float* x_gc = x_part + 640;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* tbar = reinterpret_cast<uint64_t*>(sm + OFF_TBAR);
+    uint64_t* bar2 = reinterpret_cast<uint64_t*>(sm + OFF_BAR2);
     uint32_t* slot = reinterpret_cast<uint32_t*>(sm + OFF_SLOT);
     const uint32_t sbase = smem_u32(sm);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;   // tensor-memory lane quadrant of this warp
-    const int h2 = tid >> 7;   // half: rows 32*h2.. in the elementwise stage, columns 16*h2.. elsewhere
+    const int qr = tid >> 7;   // quarter: rows 16*qr.. in the elementwise stage, columns 8*qr.. elsewhere
     const int c = tid & 127;   // key channel / state row
     constexpr int NSLICES = DV / DVS;
     const int64_t blk = blockIdx.x;
@@ -258,6 +250,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar2, 1);
         mbar_init(tbar, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_la); tma_prefetch_desc(&tm_v);
@@ -275,24 +268,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after_sync();
     const uint32_t tmem = *slot;
     const uint32_t tq = tmem + (static_cast<uint32_t>(q4 * 32) << 16);  // this warp's lane quadrant
-    uint32_t phase = 0, tphase = 0;
+    uint32_t phase = 0, phase2 = 0, tphase = 0;
 
     const int64_t v_row = static_cast<int64_t>(H) * DV;
     const int64_t state_off = (static_cast<int64_t>(n) * H + h) * DK * DV;
     const int orow = q4 * 16 + lane;  // chunk row owned in the M=64 accumulator layout (lane < 16)
-    const int scol = col0 + 16 * h2;  // first of the 16 state / output columns this thread owns
+    const int scol = col0 + 8 * qr;   // first of the 8 state / output columns this thread owns
 
-    float S[16];
+    float S[8];
     if (initial_state) {
         const float4* src = reinterpret_cast<const float4*>(initial_state + state_off + static_cast<int64_t>(c) * DV + scol);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
             const float4 x = src[i];
             S[4 * i] = x.x; S[4 * i + 1] = x.y; S[4 * i + 2] = x.z; S[4 * i + 3] = x.w;
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) S[j] = 0.f;
+        for (int j = 0; j < 8; ++j) S[j] = 0.f;
     }
     float beta_next = 0.f;
     if (tid < C && t0 + tid < t1) beta_next = to_f32(beta[(t0 + tid) * H + h]);
@@ -301,9 +294,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint64_t d_kq = sw128b32_desc(sbase + OFF_KQ, 128 * 128, 512);      // [K+|Q+]^T, MN-major
     const uint64_t d_km = sw128b32_desc(sbase + OFF_KM, 128 * 128, 512);      // (K-)^T, MN-major
     const uint64_t d_s = sw128b32_desc(sbase + OFF_S, 128 * 128, 512);        // S', MN-major
-    const uint64_t d_t = sw128_desc(sbase + OFF_T, 16, 1024);                 // T', K-major
-    const uint64_t d_v = sw128b32_desc(sbase + OFF_VD, 64 * 128, 512);        // V / Delta, MN-major
-    const uint64_t d_z = sw128b32_desc(sbase + OFF_Z, 64 * 128, 512);         // Z, MN-major
+    const uint64_t d_d = sw128b32_desc(sbase + OFF_D, 64 * 128, 512);         // Delta, MN-major
     const uint64_t d_kmt = sw128_desc(sbase + OFF_KMT, 16, 1024);             // (K-)^T, K-major
     const uint64_t d_p = sw128_desc(sbase + OFF_P, 16, 1024);                 // P, K-major
     constexpr uint64_t kQplus = (2 * 128 * 128) >> 4;                          // Q+ M-blocks
@@ -317,39 +308,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tphase ^= 1;
         tma_pending = false;
 
-        // ---- elementwise stage (thread: channel c, rows 32*h2 .. 32*h2+31)
+        // ---- elementwise stage (thread: channel c, rows 16*qr .. 16*qr+15)
         const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK);
         const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ);
         const TG* sla = reinterpret_cast<const TG*>(sm + OFF_SLA);
-        const int rb = 32 * h2;
-        float g[32];
+        const int rb = 16 * qr;
+        float g[16];
         {
             float run = 0.f;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
+            for (int r = 0; r < 16; ++r) {
                 run += (rb + r) < len ? to_f32(sla[(rb + r) * DK + c]) : 0.f;
                 g[r] = run;
             }
-            if (h2 == 0) x_part[c] = run;
+            x_part[qr * 128 + c] = run;
         }
         __syncthreads();
-        if (h2 == 1) {
-            const float off = x_part[c];
+        {
+            float off = 0.f;
+            for (int q = 0; q < qr; ++q) off += x_part[q * 128 + c];
 #pragma unroll
-            for (int r = 0; r < 32; ++r) g[r] += off;
-            x_gm[c] = g[0];
-            x_gc[c] = g[31];
-            const float g0 = len > 0 ? to_f32(sla[c]) : 0.f;
-            if (g0 - g[0] > kAnchorLimit || g[0] - g[31] > kAnchorLimit || g[0] < -kAnchorLimit)
-                raise_flag(flags, KDA_DEVFLAG_DECAY_RANGE);
+            for (int r = 0; r < 16; ++r) g[r] += off;
+            if (qr == 2) x_gm[c] = g[0];  // row 32
+            if (qr == 3) x_gc[c] = g[15];  // row 63
         }
         __syncthreads();
         const float gm = x_gm[c], gC = x_gc[c];
+        if (qr == 0 && (g[0] - gm > kAnchorLimit || gm - gC > kAnchorLimit || gm < -kAnchorLimit))
+            raise_flag(flags, KDA_DEVFLAG_DECAY_RANGE);
         const float em = expf(gm), ec = expf(gC - gm), gam = expf(gC);
-        // rows rb .. rb+31 of channel c -> row c of [K+ | Q+]^T (M-blocks h2 and 2+h2), of (K-)^T
-        // MN-major (N-block h2) and of (K-)^T K-major (K-block h2), four rows per 16-byte store
+        // rows rb .. rb+15 of channel c -> row c of [K+ | Q+]^T (M-blocks qr/2 and 2+qr/2), of (K-)^T
+        // MN-major (N-block qr/2) and of (K-)^T K-major (K-block qr/2), four rows per 16-byte store
 #pragma unroll
-        for (int r4 = 0; r4 < 32; r4 += 4) {
+        for (int r4 = 0; r4 < 16; r4 += 4) {
             float kp[4], qp[4], km[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -362,26 +353,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 qp[u] = to_tf32(qv * e);
                 km[u] = to_tf32(kv * ie);
             }
-            const int m = 32 * h2 + r4;
+            const int m = rb + r4;
             *reinterpret_cast<float4*>(sm + OFF_KQ + sw32b_off(c, m, 128)) = make_float4(kp[0], kp[1], kp[2], kp[3]);
             *reinterpret_cast<float4*>(sm + OFF_KQ + sw32b_off(c, C + m, 128)) = make_float4(qp[0], qp[1], qp[2], qp[3]);
             *reinterpret_cast<float4*>(sm + OFF_KM + sw32b_off(c, m, 128)) = make_float4(km[0], km[1], km[2], km[3]);
             *reinterpret_cast<float4*>(sm + OFF_KMT + sw128_off(c, m, 128)) = make_float4(km[0], km[1], km[2], km[3]);
         }
-        {   // S' = Diag(e^{g_m}) S0: K-row c, columns 16*h2 .. 16*h2+15 of the slice
-            float sp[16];
+        {   // S' = Diag(e^{g_m}) S0: K-row c, columns 8*qr .. 8*qr+7 of the slice
+            float sp[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) sp[j] = em * S[j];
-            st_mn8(sm, OFF_S, c, 16 * h2, 128, sp);
-            st_mn8(sm, OFF_S, c, 16 * h2 + 8, 128, sp + 8);
+            for (int j = 0; j < 8; ++j) sp[j] = em * S[j];
+            st_mn8(sm, OFF_S, c, 8 * qr, 128, sp);
         }
-        {   // V slice: thread -> (row, 8 columns)
-            const int r = tid >> 2, j0 = (tid & 3) * 8;
-            float vv[8];
+        {   // right-hand side, first part: R = Diag(beta) V  (thread -> row, 4 columns)
+            const int r = tid >> 3, j0 = (tid & 7) * 4;
             const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SV) + r * DVS + j0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) vv[i] = r < len ? __bfloat162float(sv[i]) : 0.f;
-            st_mn8(sm, OFF_VD, r, j0, 64, vv);
+            const float br = s_beta[r];  // 0 past the sequence end
+            float4 rv;
+            rv.x = r < len ? br * __bfloat162float(sv[0]) : 0.f;
+            rv.y = r < len ? br * __bfloat162float(sv[1]) : 0.f;
+            rv.z = r < len ? br * __bfloat162float(sv[2]) : 0.f;
+            rv.w = r < len ? br * __bfloat162float(sv[3]) : 0.f;
+            *reinterpret_cast<float4*>(tile(sm, OFF_R) + r * DVS + j0) = rv;
         }
         fence_async_smem();
         tc_fence_before_sync();
@@ -404,101 +397,74 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after_sync();
             const uint32_t id1 = idesc_tf32(128, 64, true, true);
             const uint32_t idz = idesc_tf32(64, DVS, true, true);
+            // MN-major tiles: K-step of 8 channels = 8 rows of 128 bytes (1024 >> 4 = 64)
 #pragma unroll
             for (int kk = 0; kk < DK / 8; ++kk) {
-                // MN-major tiles: K-step of 8 channels = 8 rows of 128 bytes (1024 >> 4 = 64)
                 const uint64_t step = static_cast<uint64_t>(kk) * 64;
-                const uint64_t akq = d_kq + step, aq = d_kq + kQplus + step;
-                const uint64_t bkm = d_km + step, bs = d_s + step;
-                mma_tf32(tmem + TM_AP, akq, bkm, id1, kk > 0);
-                mma_tf32(tmem + TM_Z, akq, bs, idz, kk > 0);
-                mma_tf32(tmem + TM_O, aq, bs, idz, kk > 0);
+                mma_tf32(tmem + TM_AP, d_kq + step, d_km + step, id1, kk > 0);
             }
-            mma_commit(bar);
+            mma_commit(bar);   // [A_raw; P]: needed first
+#pragma unroll
+            for (int kk = 0; kk < DK / 8; ++kk) {
+                const uint64_t step = static_cast<uint64_t>(kk) * 64;
+                mma_tf32(tmem + TM_Z, d_kq + step, d_s + step, idz, kk > 0);
+                mma_tf32(tmem + TM_O, d_kq + kQplus + step, d_s + step, idz, kk > 0);
+            }
+            mma_commit(bar2);  // Z, O: needed after the A readout
         }
         timed_out = !mbar_wait(bar, phase, kWaitPolls);
         phase ^= 1;
         if (__syncthreads_or(timed_out)) break;
         tc_fence_after_sync();
         {   // rows 0..63 -> A (fp32, beta-scaled, strictly lower); rows 64..127 -> P (tf32, lower)
-            float x[32];
-            tmem_ld32(tq + TM_AP + h2 * 32, x);  // M=128: row 32*q4 + lane, columns 32*h2..
+            float x[16];
+            tmem_ld16(tq + TM_AP + qr * 16, x);  // M=128: row 32*q4 + lane, columns 16*qr..
             const int row = q4 * 32 + lane;
             if (row < C) {
-                float* am = tile(sm, OFF_A);
+                float* am = tile(sm, OFF_A) + row * TP + qr * 16;
                 const float br = s_beta[row];
+                float a[16];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int i = h2 * 32 + jj;
-                    am[row * TP + i] = i < row ? br * x[jj] : 0.f;
-                }
+                for (int jj = 0; jj < 16; ++jj) a[jj] = (qr * 16 + jj) < row ? br * x[jj] : 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    reinterpret_cast<float4*>(am)[k] = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
             } else {
                 const int r = row - C;
 #pragma unroll
-                for (int jj = 0; jj < 32; jj += 4) {
-                    const int i = h2 * 32 + jj;
+                for (int jj = 0; jj < 16; jj += 4) {
+                    const int i = qr * 16 + jj;
                     st_sw4(sm, OFF_P, r, i, 64, i <= r ? x[jj] : 0.f, i + 1 <= r ? x[jj + 1] : 0.f,
                            i + 2 <= r ? x[jj + 2] : 0.f, i + 3 <= r ? x[jj + 3] : 0.f);
                 }
             }
-            float z[16];
-            tmem_ld16(tq + TM_Z + h2 * 16, z);  // M=64: row orow in lanes 0..15
-            if (lane < 16) {
-                st_mn8(sm, OFF_Z, orow, 16 * h2, 64, z);
-                st_mn8(sm, OFF_Z, orow, 16 * h2 + 8, 64, z + 8);
-            }
         }
-        tc_fence_before_sync();
-        __syncthreads();
-
-        // ---- T = (I + A)^{-1}, then T' = T Diag(beta) as an MMA operand
-        unit_lower_inverse(tile(sm, OFF_A), tile(sm, OFF_TF), tile(sm, OFF_Y));
-        {
-            const float* tf = tile(sm, OFF_TF) + (tid >> 2) * TP;
-            const int r = tid >> 2, i0 = (tid & 3) * 16;
-#pragma unroll
-            for (int i = i0; i < i0 + 16; i += 4)
-                st_sw4(sm, OFF_T, r, i, 64, tf[i] * s_beta[i], tf[i + 1] * s_beta[i + 1], tf[i + 2] * s_beta[i + 2],
-                       tf[i + 3] * s_beta[i + 3]);
-        }
-        fence_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-
-        // ---- MMA batch 2: U = T' V,  X = T' Z
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t id = idesc_tf32(64, DVS, false, true);
-#pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk) {
-                const uint64_t at = d_t + (((kk >> 2) * 64 * 128 + (kk & 3) * 32) >> 4);
-                const uint64_t bv = d_v + static_cast<uint64_t>(kk) * 64;
-                const uint64_t bz = d_z + static_cast<uint64_t>(kk) * 64;
-                mma_tf32(tmem + TM_U, at, bv, id, kk > 0);
-                mma_tf32(tmem + TM_X, at, bz, id, kk > 0);
-            }
-            mma_commit(bar);
-        }
-        timed_out = !mbar_wait(bar, phase, kWaitPolls);
-        phase ^= 1;
-        if (__syncthreads_or(timed_out)) break;
+        __syncthreads();  // A complete
+        diag_block_inverses(tile(sm, OFF_A), tile(sm, OFF_TF));
+        timed_out = !mbar_wait(bar2, phase2, kWaitPolls);
+        phase2 ^= 1;
+        if (__syncthreads_or(timed_out)) break;  // also: diagonal-block inverses complete
         tc_fence_after_sync();
-        {   // Delta = U - X  (rows in the M=64 layout, columns 16*h2..)
-            float u[16], x[16];
-            tmem_ld16(tq + TM_U + h2 * 16, u);
-            tmem_ld16(tq + TM_X + h2 * 16, x);
-            if (lane < 16) {
+        {
+            float z[8];
+            tmem_ld8(tq + TM_Z + qr * 8, z);  // M=64: row orow in lanes 0..15
+            if (lane < 16) {                  // R = Diag(beta) (V - Z)
+                float* rr = tile(sm, OFF_R) + orow * DVS + 8 * qr;
+                const float br = s_beta[orow];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) u[j] -= x[j];
-                st_mn8(sm, OFF_VD, orow, 16 * h2, 64, u);
-                st_mn8(sm, OFF_VD, orow, 16 * h2 + 8, 64, u + 8);
+                for (int j = 0; j < 8; ++j) rr[j] -= br * z[j];
             }
         }
+        tc_fence_before_sync();
+        __syncthreads();
+
+        // ---- Delta = (I + A)^{-1} R by block forward substitution, written as the tf32 Delta operand
+        block_forward_solve(tile(sm, OFF_A), tile(sm, OFF_TF), tile(sm, OFF_R), tile(sm, OFF_DL), sm, OFF_D);
         fence_async_smem();
         tc_fence_before_sync();
         __syncthreads();
 
-        // ---- MMA batch 3: Y = (K-)^T Delta (A MN-major),  O += P Delta
+        // ---- MMA batch 2: Y = (K-)^T Delta,  O += P Delta
         if (tid == 0) {
             tc_fence_after_sync();
             const uint32_t idy = idesc_tf32(128, DVS, false, true);
@@ -507,7 +473,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int kk = 0; kk < C / 8; ++kk) {
                 const uint64_t ak = d_kmt + (((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4);
                 const uint64_t ap = d_p + (((kk >> 2) * 64 * 128 + (kk & 3) * 32) >> 4);
-                const uint64_t bd = d_v + static_cast<uint64_t>(kk) * 64;
+                const uint64_t bd = d_d + static_cast<uint64_t>(kk) * 64;
                 mma_tf32(tmem + TM_Y, ak, bd, idy, kk > 0);
                 mma_tf32(tmem + TM_O, ap, bd, ido, 1);
             }
@@ -518,16 +484,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (__syncthreads_or(timed_out)) break;
         tc_fence_after_sync();
         {
-            float y[16];
-            tmem_ld16(tq + TM_Y + h2 * 16, y);  // M=128: lane = state row c
+            float y[8];
+            tmem_ld8(tq + TM_Y + qr * 8, y);  // M=128: lane = state row c
 #pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = gam * S[j] + ec * y[j];
-            float ov[16];
-            tmem_ld16(tq + TM_O + h2 * 16, ov);
+            for (int j = 0; j < 8; ++j) S[j] = gam * S[j] + ec * y[j];
+            float ov[8];
+            tmem_ld8(tq + TM_O + qr * 8, ov);
             if (lane < 16 && orow < len) {
                 const int64_t off = (c0 + orow) * v_row + static_cast<int64_t>(h) * DV + scol;
-                if (o_is_f32) store_row16<float>(static_cast<float*>(o_ptr) + off, ov);
-                else store_row16<__nv_bfloat16>(static_cast<__nv_bfloat16*>(o_ptr) + off, ov);
+                if (o_is_f32) store_row8<float>(static_cast<float*>(o_ptr) + off, ov);
+                else store_row8<__nv_bfloat16>(static_cast<__nv_bfloat16*>(o_ptr) + off, ov);
             }
         }
         tc_fence_before_sync();
@@ -540,8 +506,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (tid == 0) raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
     } else if (final_state) {
         float4* dst = reinterpret_cast<float4*>(final_state + state_off + static_cast<int64_t>(c) * DV + scol);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+        dst[0] = make_float4(S[0], S[1], S[2], S[3]);
+        dst[1] = make_float4(S[4], S[5], S[6], S[7]);
     }
     tc_fence_before_sync();
     __syncthreads();
