@@ -40,8 +40,12 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 64 * (3 * 128 + 2 * 128)
 # Decode: the fp32 state read and written once, plus q, k, v bf16, log_alpha fp32, beta fp32, o bf16.
 DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
-PREFILL_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_chunk_tc.cu", "gated_delta_rule_127_b200/csrc/kda_sm100.cuh",
-                          "gated_delta_rule_127_b200/csrc/kda_chunk_simt.cu"]
+# The prefill with a workspace is two launches: the chunk-local kernel over every chunk, then the scan.
+PREFILL_KERNELS_PER_CALL = 2
+PREFILL_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_chunk_prep.cu",
+                          "gated_delta_rule_127_b200/csrc/kda_chunk_scan.cu",
+                          "gated_delta_rule_127_b200/csrc/kda_wy.cuh", "gated_delta_rule_127_b200/csrc/kda_sm100.cuh",
+                          "gated_delta_rule_127_b200/csrc/kda_tma.h"]
 DECODE_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_decode.cu"]
 
 
@@ -424,17 +428,19 @@ def run_ours(args):
             "prefill_ms": prefill_max,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                         "kernel": "kda_chunk_fwd (prefill)", "peak_source": peak_src,
+                         "kernel": "kda_chunk_fwd (prefill: chunk_prep_kernel + chunk_scan_kernel)",
+                         "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": prefill_bytes,
                          "tensor_tflops": prefill_flops / (prefill_local * 1e-3) / 1e12,
                          "tensor_frac": prefill_flops / (prefill_local * 1e-3) / 1e12 / tf_peak},
-            "decode": {"us_per_step": 1000.0 * decode_max, "tokens_per_s": world * Bd * 1000.0 / decode_max,
+            "decode": None if args.only == "prefill" else {"us_per_step": 1000.0 * decode_max, "tokens_per_s": world * Bd * 1000.0 / decode_max,
                        "state_gbs": world * dec_bytes / (decode_max * 1e-3) / 1e9,
                        "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
                                     "frac": dec_gbs / hbm_peak, "frac_of_8tbs": dec_gbs / 8000.0,
                                     "traffic": dec_traffic, "algorithmic_bytes_per_launch": dec_bytes}},
             "e2e": e2e,
-            "gpu_launches": 2 * K,
+            "gpu_launches": K * ((0 if args.only == "decode" else PREFILL_KERNELS_PER_CALL) +
+                                 (0 if args.only == "prefill" else 1)),
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
             "cpu_baseline": cpu,
         }

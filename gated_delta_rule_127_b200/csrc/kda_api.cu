@@ -49,7 +49,7 @@ extern "C" {
 size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int dk, int dv, int chunk_size) {
     (void)chunk_size;
     if (T_total < 0 || N <= 0 || H <= 0) return 0;
-    return kda::chunk_tc_workspace_size(T_total, N, H, dk, dv);
+    return kda::chunk_wy_workspace_size(T_total, N, H, dk, dv);
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
@@ -75,8 +75,8 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
         return KDA_ERR_INVALID_ARG;
     if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
     const size_t need = kda_chunk_fwd_workspace_size(T_total, N, H, dk, dv, chunk_size);
-    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
-        return KDA_ERR_INVALID_ARG;
+    const bool have_ws = workspace != nullptr && workspace_bytes > 0;
+    if (have_ws && (workspace_bytes < need || !aligned16(workspace))) return KDA_ERR_INVALID_ARG;
 
     ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
@@ -87,7 +87,15 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     a.stream = static_cast<cudaStream_t>(stream);
     if (device_flags_ptr(&a.flags) != cudaSuccess) return KDA_ERR_CUDA;
 
-    const cudaError_t err = chunk_tc_supported(a) ? launch_chunk_tc(a) : launch_chunk_simt(a);
+    cudaError_t err;
+    if (!chunk_tc_supported(a)) {
+        err = launch_chunk_simt(a);
+    } else if (have_ws && need > 0) {
+        err = launch_chunk_prep(a);
+        if (err == cudaSuccess) err = launch_chunk_scan(a);
+    } else {
+        err = launch_chunk_tc(a);
+    }
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

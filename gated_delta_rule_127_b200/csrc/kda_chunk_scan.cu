@@ -1,0 +1,296 @@
+// kda_chunk_scan.cu -- the inter-chunk half of the chunked KDA prefill on the sm_100a tensor cores:
+// per (sequence, head), walk the chunks in order carrying the fp32 state in tensor memory.
+//
+// "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "청크 단위 병렬 알고리듬": each chunk
+// starts from the previous chunk's final state.  With the chunk record of kda_wy.cuh (computed for
+// all chunks by kda_chunk_prep.cu), chunk n is the affine map
+//   S_{n+1} = Mt_n S_n + B_n,      O_n = Qh_n S_n + Uo_n,
+// which the CTA runs transposed, so the state is the tensor cores' A operand straight from tensor
+// memory and each chunk's result is the next chunk's operand without passing through registers:
+//   S_{n+1}^T = B_n^T + S_n^T Mt_n^T    (M = dv = 128, N = 128, K = dk = 128: 16 MMAs)
+//   O_n^T     = Uo_n^T + S_n^T Qh_n^T   (M = 128, N = 64, K = 128: 16 MMAs)
+// The accumulators start from B_n^T and Uo_n^T, written into tensor memory by the data warps.  The
+// state is read by the tensor cores as tf32 (its low 13 mantissa bits ignored) and accumulated in
+// fp32; it is stored in fp32 at the end.
+//
+// Roles (320 threads): warps 0-7 fill the accumulators and store o and the final state -- warp w
+// serves value columns dv = 32 (w % 4) .. +31 (its tensor-memory lanes) and half w / 4 of the
+// accumulator columns, and holds the next chunk's share of B and Uo in registers while the current
+// chunk's MMAs run; warp 8 lane 0 brings each chunk's Mt and Qh operand tiles into a two-stage
+// shared-memory ring with bulk copies (and asks L2 for the B and Uo of the chunk after); warp 9
+// lane 0 issues the MMAs.
+// Tensor memory: three state buffers (S_n read while S_{n+1} accumulates and S_{n+2}'s B is written)
+// and two output buffers.
+#include <cuda_bf16.h>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+#include "kda_sm100.cuh"
+#include "kda_wy.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+using wy::C;
+using wy::DK;
+using wy::DV;
+
+constexpr int THREADS = 320;
+constexpr int DATA_THREADS = 256;
+constexpr int LOADER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr uint32_t kWaitPolls = 1u << 26;
+
+constexpr uint32_t STAGE_BYTES = 98304;  // Mt tile (64 KB) + Qh tile (32 KB)
+constexpr uint32_t OFF_STAGE0 = 0;
+constexpr uint32_t OFF_STAGE1 = STAGE_BYTES;
+constexpr uint32_t OFF_BARS = 2 * STAGE_BYTES;  // full[2], empty[2], chain, sinit[2], odone[2]
+constexpr uint32_t OFF_SLOT = OFF_BARS + 9 * 8;
+constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
+constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+
+constexpr uint32_t TM_S = 0;    // state buffers at 0, 128, 256
+constexpr uint32_t TM_O = 384;  // output buffers at 384, 448
+constexpr uint32_t TM_COLS = 512;
+
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, 1); }
+
+// Bounded wait that also gives up when another role has flagged an abort; a timeout flags one.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(sdst)),
+                 "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void store_o(void* o, int64_t idx, float x, bool f32) {
+    if (f32) static_cast<float*>(o)[idx] = x;
+    else static_cast<__nv_bfloat16*>(o)[idx] = __float2bfloat16_rn(x);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_state,
+                  const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H, void* __restrict__ o_ptr,
+                  int o_is_f32, float* final_state, unsigned int* flags) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
+    uint64_t* full = bars;        // [2] stage s loaded
+    uint64_t* empty = bars + 2;   // [2] stage s read by the MMAs
+    uint64_t* chain = bars + 4;   // state MMA of the latest chunk complete
+    uint64_t* sinit = bars + 5;   // [2] accumulators of chunk c (parity c & 1) initialised
+    uint64_t* odone = bars + 7;   // [2] output MMA of chunk c complete
+    uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_SLOT);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = static_cast<int>(blockIdx.x % H);
+    const int n = static_cast<int>(blockIdx.x / H);
+    int64_t t0, t1;
+    if (!wy::seq_bounds(cu_seqlens, T_total, N, n, t0, t1)) {
+        if (tid == 0) raise_flag(flags, KDA_DEVFLAG_CU_SEQLENS);
+        return;
+    }
+    const int nc = static_cast<int>((t1 - t0 + C - 1) / C);
+    const int64_t slot0 = wy::slot_base(t0, n);
+    const int64_t state_off = (static_cast<int64_t>(n) * H + h) * DK * DV;
+
+    if (tid == 0) {
+        for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
+        mbar_init(sinit, DATA_THREADS);
+        mbar_init(sinit + 1, DATA_THREADS);
+        mbar_init(odone, 1);
+        mbar_init(odone + 1, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(slot_tm, TM_COLS);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *slot_tm;
+
+    if (warp < 8) {
+        // ---------------- data warps: lane = value column dv, g = half of the accumulator columns
+        const int dv = 32 * (warp & 3) + lane;
+        const int g = warp >> 2;
+        const uint32_t tq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        {   // S_0^T into state buffer 0 (rows i = 64 g .. 64 g + 63 of S_0)
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int i0 = 64 * g + 32 * jj;
+                float v[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    v[e] = initial_state ? initial_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] : 0.f;
+                tmem_st32(tq + TM_S + i0, v);
+            }
+            tmem_st_wait();
+        }
+        auto emit_o = [&](int c) {  // tokens 32 g .. 32 g + 31 of O_c^T (output buffer c & 1) -> o
+            const int64_t c0 = t0 + static_cast<int64_t>(c) * C;
+            const int len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
+            float x[32];
+            tmem_ld32(tq + TM_O + 64 * (c & 1) + 32 * g, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int t = 32 * g + e;
+                if (t < len) store_o(o_ptr, ((c0 + t) * H + h) * DV + dv, x[e], o_is_f32 != 0);
+            }
+        };
+        // this thread's share of chunk c's B^T (rows i = 64 g .. +63) and Uo^T (tokens 32 g .. +31)
+        float4 pb[16], pu[8];
+        auto fetch = [&](int c) {
+            const float4* rec =
+                reinterpret_cast<const float4*>(ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES);
+            const float4* gB = rec + wy::REC_B / 16 + (16 * g) * 128 + dv;
+            const float4* gU = rec + wy::REC_UO / 16 + (8 * g) * 128 + dv;
+#pragma unroll
+            for (int s = 0; s < 16; ++s) pb[s] = __ldcs(gB + s * 128);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) pu[s] = __ldcs(gU + s * 128);
+        };
+        auto put32 = [&](uint32_t taddr, const float4* p) {
+            float v[32];
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                v[4 * s] = p[s].x; v[4 * s + 1] = p[s].y; v[4 * s + 2] = p[s].z; v[4 * s + 3] = p[s].w;
+            }
+            tmem_st32(taddr, v);
+        };
+        bool ok = true;
+        if (nc > 0) fetch(0);
+        for (int c = 0; c < nc && ok; ++c) {
+            if (c >= 2) {
+                ok = wait_or_abort(odone + (c & 1), ((c - 2) >> 1) & 1, abort);
+                if (!ok) break;
+                tc_fence_after_sync();
+                emit_o(c - 2);
+            }
+            const uint32_t sb = TM_S + 128 * ((c + 1) % 3) + 64 * g;
+            put32(tq + sb, pb);
+            put32(tq + sb + 32, pb + 8);
+            put32(tq + TM_O + 64 * (c & 1) + 32 * g, pu);
+            tmem_st_wait();
+            tc_fence_before_sync();
+            mbar_arrive(sinit + (c & 1));
+            if (c + 1 < nc) fetch(c + 1);
+        }
+        for (int c = nc - 2 < 0 ? 0 : nc - 2; c < nc && ok; ++c) {
+            ok = wait_or_abort(odone + (c & 1), (c >> 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after_sync();
+            emit_o(c);
+        }
+        if (ok && final_state) {  // after the last output MMA, the last state MMA is complete too
+            const uint32_t sb = TM_S + 128 * (nc % 3);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int i0 = 64 * g + 32 * jj;
+                float x[32];
+                tmem_ld32(tq + sb + i0, x);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) final_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = x[e];
+            }
+        }
+    } else if (warp == LOADER_WARP) {
+        // ---------------- loader: chunk c's Mt and Qh tiles into stage c & 1
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = 0; c < nc; ++c) {
+                const int s = c & 1;
+                if (c >= 2 && !wait_or_abort(empty + s, ((c - 2) >> 1) & 1, abort)) break;
+                const unsigned char* rec = ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES;
+                unsigned char* stage = sm + (s ? OFF_STAGE1 : OFF_STAGE0);
+                mbar_arrive_expect_tx(full + s, STAGE_BYTES);
+#pragma unroll
+                for (int b = 0; b < 4; ++b) bulk_load(stage + 16384 * b, rec + wy::REC_M + 16384 * b, 16384, full + s);
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+                    bulk_load(stage + 65536 + 16384 * b, rec + wy::REC_Q + 16384 * b, 16384, full + s);
+                if (c + 2 < nc) {  // B and Uo of chunk c + 2: the data warps fetch them a chunk later
+                    const unsigned char* r2 = ws + (static_cast<size_t>(slot0 + c + 2) * H + h) * wy::REC_BYTES;
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r2 + wy::REC_B),
+                                 "r"(wy::REC_BYTES - wy::REC_B)
+                                 : "memory");
+                }
+                issued = c + 1;
+            }
+            if (*abort) {  // leave no copy into shared memory behind: wait (bounded) for the last two
+                for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
+                    mbar_wait(full + (c & 1), (c >> 1) & 1, kWaitPolls);
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t sbase = smem_u32(sm);
+            constexpr uint32_t id_s = idesc_tf32(128, 128, false, false);
+            constexpr uint32_t id_o = idesc_tf32(128, 64, false, false);
+            int committed = 0;
+            for (int c = 0; c < nc; ++c) {
+                const int s = c & 1;
+                if (!wait_or_abort(full + s, (c >> 1) & 1, abort)) break;
+                if (!wait_or_abort(sinit + s, (c >> 1) & 1, abort)) break;
+                if (c >= 1 && !wait_or_abort(chain, (c - 1) & 1, abort)) break;
+                tc_fence_after_sync();
+                const uint32_t st = sbase + (s ? OFF_STAGE1 : OFF_STAGE0);
+                const uint64_t bm = sw128_desc(st, 16, 1024);
+                const uint64_t bq = sw128_desc(st + 65536, 16, 1024);
+                const uint32_t a_s = tmem + TM_S + 128 * (c % 3);
+                const uint32_t d_s = tmem + TM_S + 128 * ((c + 1) % 3);
+                const uint32_t d_o = tmem + TM_O + 64 * s;
+#pragma unroll
+                for (int kk = 0; kk < DK / 8; ++kk)
+                    mma_tf32_ts(d_s, a_s + 8 * kk, bm + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), id_s, 1);
+                mma_commit(chain);
+#pragma unroll
+                for (int kk = 0; kk < DK / 8; ++kk)
+                    mma_tf32_ts(d_o, a_s + 8 * kk, bq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_o, 1);
+                mma_commit(empty + s);
+                mma_commit(odone + s);
+                committed = c + 1;
+            }
+            if (*abort && committed > 0)  // let the tensor cores finish before the memory is released
+                mbar_wait(odone + ((committed - 1) & 1), ((committed - 1) >> 1) & 1, kWaitPolls);
+        }
+        __syncwarp();
+    }
+
+    __syncthreads();
+    if (tid == 0 && *abort) raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_scan(const ChunkArgs& a) {
+    cudaError_t err =
+        cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    const int64_t blocks = static_cast<int64_t>(a.N) * a.H;
+    chunk_scan_kernel<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
+        static_cast<const unsigned char*>(a.workspace), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
+        a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

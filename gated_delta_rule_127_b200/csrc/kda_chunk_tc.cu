@@ -572,6 +572,5 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a) {
     return a.dtype_gate == KDA_FP32 ? launch_typed<float>(a) : launch_typed<__nv_bfloat16>(a);
 }
 
-size_t chunk_tc_workspace_size(int64_t, int, int, int, int) { return 0; }
 
 }  // namespace kda

@@ -1,0 +1,40 @@
+// kda_tma.h -- host-side TMA descriptors for libkda's [T, H, d] inputs: a 3-D tensor map with d
+// innermost, then heads, then tokens, so one box is `box0` consecutive channels of one head for
+// `box2` consecutive tokens.  The driver entry point is looked up once through the runtime.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+namespace kda {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tma_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// d0 = channels, d1 = heads, d2 = tokens; box {box0, 1, box2}.  Out-of-range tokens read as zero.
+inline bool tma_encode_thd(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, uint64_t d0,
+                           uint64_t d1, uint64_t d2, uint32_t box0, uint32_t box2, CUtensorMapSwizzle swz) {
+    auto fn = tma_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+    const cuuint32_t box[3] = {box0, 1, box2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace kda

@@ -112,12 +112,14 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: 
                   chunk_size: int = 64, o: Optional[torch.Tensor] = None,
                   final_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
                   dtype_o: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
-                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                  use_workspace: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """KDA chunked prefill over a packed batch (see kda_chunk_fwd in include/kda.h).
 
     q, k, log_alpha [T, H, dk]; v [T, H, dv]; beta [T, H]; initial_state [N, H, dk, dv] fp32 or None;
     cu_seqlens [N+1] int32 CUDA tensor, or None with `num_seqs` equal-length sequences (default 1).
     Returns (o [T, H, dv], final_state [N, H, dk, dv] fp32 or None).
+    A workspace of kda_chunk_fwd_workspace_size bytes is allocated when none is given; with
+    use_workspace=False none is passed and the library runs its workspace-free kernel.
     """
     lib = load_library()
     if q.dim() != 3 or k.shape != q.shape or log_alpha.shape != q.shape or v.dim() != 3 or beta.dim() != 2:
@@ -150,7 +152,9 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: 
     _check_cuda(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, initial_state=initial_state,
                      cu_seqlens=cu_seqlens, o=o, final_state=final_state, workspace=workspace), device)
     need = int(lib.kda_chunk_fwd_workspace_size(T, N, H, dk, dv, chunk_size))
-    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+    if not use_workspace:
+        workspace = None
+    elif need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(device):

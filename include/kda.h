@@ -90,11 +90,16 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int d
  *   T_total >= 0, N >= 1, H >= 1, dk, dv in {64, 128}, chunk_size == 64
  *   o           [T_total, H, dv]  dtype_o          output (may not alias an input)
  *   final_state [N, H, dk, dv]    fp32 or NULL     NULL = not written; may alias initial_state
- *   workspace   device scratch of workspace_bytes >= kda_chunk_fwd_workspace_size(...), or NULL
- *               when that size is 0.
+ *   workspace   device scratch, 16-byte aligned, workspace_bytes >= kda_chunk_fwd_workspace_size(...);
+ *               or NULL / 0 bytes.  Owned by the caller; its contents on entry do not matter and are
+ *               garbage on exit.  A non-NULL workspace smaller than the size returns
+ *               KDA_ERR_INVALID_ARG.
  *
- * Path: dtype_qkv == KDA_FP32 runs the fp32 CUDA-core path (every product in fp32); KDA_BF16 with
- * dk = dv = 128 runs the tensor-core path (bf16 operands, fp32 accumulation and fp32 state).
+ * Path: dtype_qkv == KDA_FP32 runs the fp32 CUDA-core path (every product in fp32; no workspace
+ * used).  KDA_BF16 with dk = dv = 128 runs on the tensor cores (tf32 products, fp32 accumulation and
+ * fp32 state): with the workspace, a chunk-local kernel over all chunks at once followed by a scan
+ * over each sequence's chunks (about 3 KB of workspace per token and head); without it, one kernel
+ * per (sequence, head, 32-column slice of dv) that does both, slower.
  */
 KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          const void* log_alpha, const void* beta,

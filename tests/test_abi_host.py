@@ -63,6 +63,8 @@ def _chunk(lib, **kw):
     (dict(cu=FAKE + 2), kda.KDA_ERR_INVALID_ARG),
     (dict(dq=7), kda.KDA_ERR_INVALID_ARG),
     (dict(do=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(ws=FAKE, wsb=16), kda.KDA_ERR_INVALID_ARG),      # a workspace, but smaller than the size
+    (dict(ws=FAKE + 8, wsb=1 << 40), kda.KDA_ERR_INVALID_ARG),  # misaligned workspace
 ])
 def test_chunk_fwd_rejects_on_host(lib, kw, expect):
     assert _chunk(lib, **kw) == expect
@@ -91,6 +93,9 @@ def test_decode_step_rejects_on_host(lib, kw, expect):
 
 
 def test_workspace_size_is_a_pure_host_function(lib):
-    assert kda.kda_chunk_fwd_workspace_size(0, 1, 1, 128, 128) >= 0
-    assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) >= 0
+    assert kda.kda_chunk_fwd_workspace_size(0, 1, 1, 128, 128) == 0
     assert lib.kda_chunk_fwd_workspace_size(-1, 1, 1, 128, 128, 64) == 0
+    assert kda.kda_chunk_fwd_workspace_size(4096, 1, 1, 64, 64) == 0   # the fp32 / d=64 paths use none
+    # one 192 KB record per (chunk slot, head); slots = T / 64 + N + 1
+    assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) == (512 + 2) * 32 * 196608
+    assert kda.kda_chunk_fwd_workspace_size(1000, 3, 2, 128, 128) == (15 + 4) * 2 * 196608

@@ -23,16 +23,16 @@ def _built():
     kda.load_library()
 
 
-def _run(inp, dtype_o=torch.float32):
+def _run(inp, dtype_o=torch.float32, use_workspace=True):
     o, sf = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, inp.cu_seqlens,
-                              dtype_o=dtype_o)
+                              dtype_o=dtype_o, use_workspace=use_workspace)
     st, flags = kda.kda_get_device_status()
     assert st == kda.KDA_OK and flags == 0, (st, flags)
     return o, sf
 
 
-def _check_full(inp, dtype):
-    o, sf = _run(inp)
+def _check_full(inp, dtype, use_workspace=True):
+    o, sf = _run(inp, use_workspace=use_workspace)
     o_ref, s_ref = oracle_full(inp)
     eo, es = o_err(to_np(o), o_ref), s_err(to_np(sf), s_ref)
     tol_o, tol_s = TOL[dtype]
@@ -57,6 +57,19 @@ def test_ragged_varlen(dtype, dk, dv):
     lengths = [1, 63, 64, 65, 130, 0, 200, 7]
     inp = gen.make_prefill(lengths, 3, dk, dv, dtype=dtype, init_state=True, seed=11, device=DEV)
     _check_full(inp, dtype)
+
+
+@pytest.mark.parametrize("case", ["ragged", "bf16_gates", "b2_h4_t2048"])
+def test_workspace_free_kernel(case):
+    """Without a workspace the bf16 dk = dv = 128 path runs the single fused kernel."""
+    if case == "ragged":
+        inp = gen.make_prefill([1, 63, 64, 65, 130, 0, 200, 7], 3, 128, 128, init_state=True, seed=21, device=DEV)
+    elif case == "bf16_gates":
+        inp = gen.make_prefill([300, 77], 2, 128, 128, gate_dtype=torch.bfloat16, init_state=True, seed=22,
+                               device=DEV)
+    else:
+        inp = gen.make_workload("prefill_b2_h4_t2048", device=DEV)
+    _check_full(inp, torch.bfloat16, use_workspace=False)
 
 
 def test_bf16_gates():
