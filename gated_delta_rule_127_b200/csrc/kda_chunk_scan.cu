@@ -155,12 +155,12 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
         auto fetch = [&](int c) {
             const float4* rec =
                 reinterpret_cast<const float4*>(ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES);
-            const float4* gB = rec + wy::REC_B / 16 + (16 * g) * 128 + dv;
-            const float4* gU = rec + wy::REC_UO / 16 + (8 * g) * 128 + dv;
+            const float4* gB = rec + wy::REC_B / 16 + (16 * g) * 128;
+            const float4* gU = rec + wy::REC_UO / 16 + (8 * g) * 128;
 #pragma unroll
-            for (int s = 0; s < 16; ++s) pb[s] = __ldcs(gB + s * 128);
+            for (int s = 0; s < 16; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) pu[s] = __ldcs(gU + s * 128);
+            for (int s = 0; s < 8; ++s) pu[s] = __ldcs(gU + s * 128 + dv);
         };
         auto put32 = [&](uint32_t taddr, const float4* p) {
             float v[32];
@@ -220,11 +220,10 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
 #pragma unroll
                 for (int b = 0; b < 2; ++b)
                     bulk_load(stage + 65536 + 16384 * b, rec + wy::REC_Q + 16384 * b, 16384, full + s);
-                if (c + 2 < nc) {  // B and Uo of chunk c + 2: the data warps fetch them a chunk later
-                    const unsigned char* r2 = ws + (static_cast<size_t>(slot0 + c + 2) * H + h) * wy::REC_BYTES;
-                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r2 + wy::REC_B),
-                                 "r"(wy::REC_BYTES - wy::REC_B)
-                                 : "memory");
+                if (c + 3 < nc) {  // the record three chunks ahead into L2
+                    const unsigned char* r3 = ws + (static_cast<size_t>(slot0 + c + 3) * H + h) * wy::REC_BYTES;
+                    for (uint32_t off = 0; off < wy::REC_BYTES; off += 16384)
+                        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r3 + off), "r"(16384) : "memory");
                 }
                 issued = c + 1;
             }
@@ -238,8 +237,8 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t sbase = smem_u32(sm);
-            constexpr uint32_t id_s = idesc_tf32(128, 128, false, false);
-            constexpr uint32_t id_o = idesc_tf32(128, 64, false, false);
+            constexpr uint32_t id_s = idesc_tf32(128, 128, false, true);
+            constexpr uint32_t id_o = idesc_tf32(128, 64, false, true);
             int committed = 0;
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
@@ -248,18 +247,18 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
                 if (c >= 1 && !wait_or_abort(chain, (c - 1) & 1, abort)) break;
                 tc_fence_after_sync();
                 const uint32_t st = sbase + (s ? OFF_STAGE1 : OFF_STAGE0);
-                const uint64_t bm = sw128_desc(st, 16, 1024);
-                const uint64_t bq = sw128_desc(st + 65536, 16, 1024);
+                const uint64_t bm = sw128b32_desc(st, 128 * 128, 512);           // Mt, MN-major
+                const uint64_t bq = sw128b32_desc(st + 65536, 128 * 128, 512);   // Qh, MN-major
                 const uint32_t a_s = tmem + TM_S + 128 * (c % 3);
                 const uint32_t d_s = tmem + TM_S + 128 * ((c + 1) % 3);
                 const uint32_t d_o = tmem + TM_O + 64 * s;
 #pragma unroll
-                for (int kk = 0; kk < DK / 8; ++kk)
-                    mma_tf32_ts(d_s, a_s + 8 * kk, bm + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), id_s, 1);
+                for (int kk = 0; kk < DK / 8; ++kk)  // K-step: 8 K-rows of 128 bytes
+                    mma_tf32_ts(d_s, a_s + 8 * kk, bm + static_cast<uint64_t>(kk) * 64, id_s, 1);
                 mma_commit(chain);
 #pragma unroll
                 for (int kk = 0; kk < DK / 8; ++kk)
-                    mma_tf32_ts(d_o, a_s + 8 * kk, bq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_o, 1);
+                    mma_tf32_ts(d_o, a_s + 8 * kk, bq + static_cast<uint64_t>(kk) * 64, id_o, 1);
                 mma_commit(empty + s);
                 mma_commit(odone + s);
                 committed = c + 1;
