@@ -15,8 +15,9 @@
 //   [W | U] = T [beta K e^G | beta V]                                    MMA 2
 //   P W,  Kt^T W,  B^T = U^T Kt,  Uo^T = U^T P^T                          MMAs 3-6
 //   Mt = Diag(e^{g_C}) - Kt^T W,  Qh = Q e^G - P W
-// B and Uo are formed transposed so that the accumulator lane is the value column, which lets every
-// part of the record go from registers straight to memory in whole contiguous runs.
+// B and Uo are formed transposed so that the accumulator lane is the value column: they go from
+// registers straight to memory in contiguous runs.  Mt and Qh are staged in shared memory as the
+// scan's operand tiles and written with bulk copies.
 // The anchor split e^{g_r - g_i} = e^{g_r - g_m} e^{g_m - g_i} keeps every factor that can exceed 1
 // below e^80 while the chunk's log-decay stays within 80 of g_m at both ends ("일반 DPLR보다 줄어든
 // 연산량" on the same page notes that fine-grained decay makes intra-chunk division delicate);
@@ -24,8 +25,7 @@
 // accumulation (operands rounded to tf32 when written); B and Uo are stored in fp32.
 //
 // Persistent CTAs of 512 threads, one per SM, each taking (chunk slot, head) tasks in turn.  The next
-// task's input tiles are requested into L2 when a task starts and loaded into shared memory while the
-// task's last results are being stored.  Elementwise pass: thread t owns key
+// task's input tiles are loaded into shared memory while the task's results are being stored.  Elementwise pass: thread t owns key
 // channel c = 32 (w % 4) + lane (its tensor-memory lane, w = warp) and rows 16 (w / 4) .. +15, so the
 // cumulative sum runs down a column in registers.  Row pass and accumulator read-outs: the warp's
 // lane quadrant gives the row, w / 4 the column quarter.
@@ -59,17 +59,21 @@ constexpr uint32_t OFF_KM = 81920;     // K- K-major: rows s (64) x K c (128), M
 constexpr uint32_t OFF_B8 = 114688;    // [beta K e^G | beta V] K-major: rows n (256) x K s (64), MMA 2's B;
                                        //   then [W | U] MN-major: K-rows s (64) x N n (256), operand of MMAs 3-6
 constexpr uint32_t OFF_KT = 180224;    // Kt^T K-major: rows c (128) x K s (64), A of MMA 4 and B of MMA 5
-constexpr uint32_t OFF_MISC = 212992;  // beta[64], quarter-column sums[4][128], g_m, g_C, e^{g_m}, e^{g_C} [128]
-constexpr uint32_t OFF_X = 217344;     // 32 x 32 fp32 scratch for the inverse
-constexpr uint32_t OFF_TASK = 221440;  // two TaskInfo slots (this task, the next)
-constexpr uint32_t OFF_BARS = 221504;  // mbarriers: TMA, MMA 1-2, MMA 3, MMAs 4-6; then the TMEM base address
-constexpr uint32_t SMEM_USED = 221544;
+constexpr uint32_t OFF_MISC = 212992;  // beta[2][64] (this task, the next), quarter-column sums[4][128],
+                                       //   g_m, g_C, e^{g_m}, e^{g_C} [128]
+constexpr uint32_t OFF_X = 217600;     // 32 x 32 fp32 scratch for the inverse
+constexpr uint32_t OFF_TASK = 221696;  // three Task slots (this task, the next, the one after)
+constexpr uint32_t OFF_BARS = 221792;  // mbarriers: TMA, MMAs 1-2, MMAs 3-6; then the TMEM base address
+constexpr uint32_t SMEM_USED = 221832;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 // after MMA 1 (k, v staging and K- are dead):
 constexpr uint32_t OFF_A = 49152;      // A fp32 [64][TP]
 constexpr uint32_t OFF_T32 = 65536;    // T fp32 [64][TP]
 constexpr uint32_t OFF_TIMG = 81920;   // T K-major rows r x K s (64), MMA 2's A
 constexpr uint32_t OFF_P = 98304;      // P K-major rows t x K s (64), A of MMA 3 and B of MMA 6
+// record staging once MMAs 3-6 are done, outside the input staging so the next task's tiles can load:
+constexpr uint32_t STG_M = OFF_B8;     // Mt K-major rows i x K j (128), 64 KB
+constexpr uint32_t STG_Q = OFF_KT;     // Qh K-major rows t x K j (128), 32 KB
 
 // ---- tensor memory columns (512 allocated)
 constexpr uint32_t TM_A1 = 0;     // [K+; Q+], 128 x 128, MMA 1's A
@@ -104,55 +108,76 @@ __device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {
     }
 }
 
-__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int x, int y, int z) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap), "r"(x), "r"(y),
-                 "r"(z)
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+                 "r"(bytes)
                  : "memory");
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
-// Task = (chunk slot, head), slot-major so consecutive tasks share the same tokens.  Resolves the
-// slot to its sequence and first token; false for slots no chunk uses (or a malformed cu_seqlens,
-// which also raises the flag).
+// Task = (chunk slot, head), slot-major so consecutive tasks share the same tokens.
 struct Task {
-    int64_t id;   // task index, or -1: no task left
+    int64_t id;   // slot * H + head, or -1: no task left
     int64_t c0;   // first token
     unsigned char* rec;
     int h, len;
 };
-__device__ __forceinline__ bool resolve_task(int64_t task, const int32_t* cu, int64_t T_total, int N, int H,
-                                             unsigned char* ws, unsigned int* flags, Task& t) {
-    const int64_t slot = task / H;
-    t.id = task;
-    t.h = static_cast<int>(task % H);
-    auto cu_at = [&](int n) -> int64_t {
-        return cu ? static_cast<int64_t>(cu[n]) : static_cast<int64_t>(n) * (T_total / N);
-    };
-    int lo = 0, hi = N - 1;  // the last sequence whose first slot is <= slot
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (wy::slot_base(cu_at(mid), mid) <= slot) lo = mid;
-        else hi = mid - 1;
+
+// Walks a CTA's tasks blockIdx.x, blockIdx.x + gridDim.x, ... in order.  Slots never decrease along
+// the walk, so the sequence holding the current slot is found by stepping forward from the last one
+// (no division or search per task).  Slots no chunk uses are skipped; a malformed cu_seqlens raises
+// the flag and skips the slot.
+struct TaskWalker {
+    const int32_t* cu;
+    int64_t T_total, L, nslots, slot, step_slot;
+    unsigned char* ws;
+    unsigned int* flags;
+    int N, H, h, step_h, n;
+
+    __device__ __forceinline__ int64_t cu_at(int i) const {
+        return cu ? static_cast<int64_t>(cu[i]) : static_cast<int64_t>(i) * L;
     }
-    int64_t t0, t1;
-    if (!wy::seq_bounds(cu, T_total, N, lo, t0, t1)) {
-        raise_flag(flags, KDA_DEVFLAG_CU_SEQLENS);
-        return false;
+    __device__ __forceinline__ void init(const int32_t* cu_, int64_t T_total_, int N_, int H_, unsigned char* ws_,
+                                         unsigned int* flags_) {
+        cu = cu_; T_total = T_total_; N = N_; H = H_; ws = ws_; flags = flags_;
+        L = T_total / N;
+        nslots = wy::num_slots(T_total, N);
+        slot = blockIdx.x / H;
+        h = static_cast<int>(blockIdx.x % H);
+        step_slot = gridDim.x / H;
+        step_h = static_cast<int>(gridDim.x % H);
+        n = 0;
     }
-    t.c0 = t0 + (slot - wy::slot_base(t0, lo)) * C;
-    if (t.c0 < t0 || t.c0 >= t1) return false;
-    t.len = static_cast<int>((t1 - t.c0) < C ? (t1 - t.c0) : C);
-    t.rec = ws + (static_cast<size_t>(slot) * H + t.h) * wy::REC_BYTES;
-    return true;
-}
-// The first task from `from` on (stepping by `step`) that holds a chunk; id = -1 when none is left.
-__device__ __forceinline__ Task next_task(int64_t from, int64_t step, int64_t ntasks, const int32_t* cu,
-                                          int64_t T_total, int N, int H, unsigned char* ws, unsigned int* flags) {
-    Task t;
-    for (int64_t x = from; x < ntasks; x += step)
-        if (resolve_task(x, cu, T_total, N, H, ws, flags, t)) return t;
-    t.id = -1;
-    return t;
-}
+    __device__ __forceinline__ void advance() {
+        h += step_h;
+        slot += step_slot;
+        if (h >= H) { h -= H; ++slot; }
+    }
+    // The next task that holds a chunk (id = -1 when none is left); moves past it.
+    __device__ __forceinline__ Task next() {
+        Task t;
+        for (; slot < nslots; advance()) {
+            while (n + 1 < N && wy::slot_base(cu_at(n + 1), n + 1) <= slot) ++n;
+            const int64_t t0 = cu_at(n), t1 = cu_at(n + 1);
+            if (cu && (t0 < 0 || t1 < t0 || t1 > T_total || (n == 0 && t0 != 0) || (n == N - 1 && t1 != T_total))) {
+                raise_flag(flags, KDA_DEVFLAG_CU_SEQLENS);
+                continue;
+            }
+            const int64_t c0 = t0 + (slot - wy::slot_base(t0, n)) * C;
+            if (c0 < t0 || c0 >= t1) continue;
+            t.id = slot * H + h;
+            t.c0 = c0;
+            t.h = h;
+            t.len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
+            t.rec = ws + (static_cast<size_t>(slot) * H + h) * wy::REC_BYTES;
+            advance();
+            return t;
+        }
+        t.id = -1;
+        return t;
+    }
+};
 
 // T = (I + A)^{-1} for A strictly lower (fp32, row stride TP) into tm, fully written (zero above the
 // diagonal).  xs: 1024 floats of scratch.  The 16 x 16 diagonal blocks by forward substitution, then
@@ -165,10 +190,21 @@ __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, f
             float t[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float acc = (r == j) ? 1.f : 0.f;
+                float a[16];  // row r of the block (columns < r are used), broadcast reads
 #pragma unroll
-                for (int i = 0; i < r; ++i) acc -= am[(b + r) * TP + b + i] * t[i];
-                t[r] = (r >= j) ? acc : 0.f;
+                for (int i4 = 0; i4 < 16; i4 += 4) {
+                    if (i4 < r) {
+                        const float4 v = *reinterpret_cast<const float4*>(am + (b + r) * TP + b + i4);
+                        a[i4] = v.x; a[i4 + 1] = v.y; a[i4 + 2] = v.z; a[i4 + 3] = v.w;
+                    }
+                }
+                float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int i = 0; i < r; ++i) {
+                    if (i & 1) acc1 -= a[i] * t[i];
+                    else acc0 -= a[i] * t[i];
+                }
+                t[r] = (r >= j) ? acc0 + acc1 : 0.f;
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) tm[(b + r) * TP + b + j] = t[r];
@@ -248,75 +284,69 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;   // tensor-memory lane quadrant
     const int qr = warp >> 2;  // row quarter (elementwise pass) / column quarter (read-outs)
-    const int64_t ntasks = wy::num_slots(T_total, N) * H;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(sm);
-    float* s_beta = reinterpret_cast<float*>(sm + OFF_MISC);
-    float* x_part = s_beta + 64;   // [4][128]
+    float* s_beta2 = reinterpret_cast<float*>(sm + OFF_MISC);  // [2][64], by task parity
+    float* x_part = s_beta2 + 128;  // [4][128]
     float* x_gm = x_part + 512;
     float* x_gc = x_gm + 128;
     float* x_egm = x_gc + 128;
     float* x_gam = x_egm + 128;
     float* xs = reinterpret_cast<float*>(sm + OFF_X);
-    Task* slots = reinterpret_cast<Task*>(sm + OFF_TASK);  // [it & 1]: this task; [(it + 1) & 1]: the next
+    Task* slots = reinterpret_cast<Task*>(sm + OFF_TASK);  // ring of 3: this task, the next, the one after
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_tma + 1;   // MMAs 1 and 2
-    uint64_t* bar_pw = bar_tma + 2;    // MMA 3
-    uint64_t* bar_rest = bar_tma + 3;  // MMAs 4-6
+    uint64_t* bar_rest = bar_tma + 2;  // MMAs 3-6
     uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 32);
 
     constexpr uint32_t kGateBytes = C * DK * sizeof(TG);
     constexpr uint32_t kStageBytes = 3 * C * DK * 2 + kGateBytes;
-    // The task's q, k, v and log_alpha tiles: into the staging buffers (bar_tma), or only into L2.
-    auto issue_loads = [&](const Task& t, bool to_l2) {
-        const int y = static_cast<int>(t.c0);
-        const CUtensorMap* maps[3] = {&tm_k, &tm_q, &tm_v};
-        const uint32_t dst[3] = {OFF_SK, OFF_SQ, OFF_SV};
-        if (!to_l2) mbar_arrive_expect_tx(bar_tma, kStageBytes);
-#pragma unroll
-        for (int m = 0; m < 3; ++m)
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                if (to_l2) tma_prefetch_l2_3d(maps[m], 64 * b, t.h, y);
-                else tma_load_3d(sm + dst[m] + 8192 * b, maps[m], 64 * b, t.h, y, bar_tma);
-            }
-        if (sizeof(TG) == 4) {
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                if (to_l2) tma_prefetch_l2_3d(&tm_g, 32 * b, t.h, y);
-                else tma_load_3d(sm + OFF_G + b * 8192, &tm_g, 32 * b, t.h, y, bar_tma);
-            }
+    // Box j of the task's q, k, v and log_alpha tiles into the staging buffers (completion on bar_tma,
+    // whose expected byte count kStageBytes is set once per task).  The boxes are issued by different
+    // warps so that no thread serialises all of them.
+    constexpr int kLoads = sizeof(TG) == 4 ? 10 : 8;
+    auto load_box = [&](const Task& t, int j) {
+        const int y = static_cast<int>(t.c0), hh = t.h;
+        const CUtensorMap* m = j < 2 ? &tm_k : j < 4 ? &tm_q : j < 6 ? &tm_v : &tm_g;
+        uint32_t dst;
+        int x;
+        if (j < 6) {
+            dst = (j < 2 ? OFF_SK : j < 4 ? OFF_SQ : OFF_SV) + 8192 * (j & 1);
+            x = 64 * (j & 1);
+        } else if (sizeof(TG) == 4) {
+            dst = OFF_G + 8192 * (j - 6);
+            x = 32 * (j - 6);
         } else {
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                if (to_l2) tma_prefetch_l2_3d(&tm_g, 64 * b, t.h, y);
-                else tma_load_3d(sm + OFF_G + 16384 + b * 8192, &tm_g, 64 * b, t.h, y, bar_tma);
-            }
+            dst = OFF_G + 16384 + 8192 * (j - 6);
+            x = 64 * (j - 6);
         }
+        tma_load_3d(sm + dst, m, x, hh, y, bar_tma);
     };
 
     uint32_t loads_issued = 0;  // thread 0: staging loads issued (bar_tma phases)
+    TaskWalker walker;          // thread 0's
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
-        mbar_init(bar_pw, 1);
         mbar_init(bar_rest, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_g);
-        const Task t0 = next_task(blockIdx.x, gridDim.x, ntasks, cu_seqlens, T_total, N, H, ws, flags);
+        walker.init(cu_seqlens, T_total, N, H, ws, flags);
+        const Task t0 = walker.next();
         Task t1;
         t1.id = -1;
         if (t0.id >= 0) {
-            issue_loads(t0, false);
+            mbar_arrive_expect_tx(bar_tma, kStageBytes);
+            for (int j = 0; j < kLoads; ++j) load_box(t0, j);
             ++loads_issued;
-            t1 = next_task(t0.id + gridDim.x, gridDim.x, ntasks, cu_seqlens, T_total, N, H, ws, flags);
-            if (t1.id >= 0) issue_loads(t1, true);
+            t1 = walker.next();
         }
         slots[0] = t0;
         slots[1] = t1;
+        slots[2].id = -1;
     }
     if (warp == 0) tmem_alloc(slot_tm, TM_COLS);
     tc_fence_before_sync();
@@ -326,13 +356,23 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tq = tmem + (static_cast<uint32_t>(q4 * 32) << 16);  // this warp's lane quadrant
     const int c = 32 * q4 + lane;  // key channel (elementwise pass) and tensor-memory lane
     bool failed = false;
+    // beta of a task into s_beta2[parity] (threads 64..127; later read only after a barrier)
+    auto load_beta = [&](const Task& t, uint32_t parity) {
+        const int r = tid - 64;
+        if (r >= 0 && r < C && t.id >= 0)
+            s_beta2[64 * parity + r] = r < t.len ? to_f32(beta[(t.c0 + r) * H + t.h]) : 0.f;
+    };
+    load_beta(slots[0], 0);  // (slots are written by thread 0 before the barrier above)
+    __syncthreads();
 
-    for (uint32_t it = 0;; ++it) {  // tasks this CTA has taken: the barriers' phase parities follow from it
-        const Task tk = slots[it & 1];
+    int cur = 0;  // slot of this task in the ring of three
+    for (uint32_t it = 0;; ++it, cur = cur == 2 ? 0 : cur + 1) {  // `it`: tasks taken; phase parities follow from it
+        const int nxt = cur == 2 ? 0 : cur + 1, aft = nxt == 2 ? 0 : nxt + 1;
+        const Task tk = slots[cur];
         if (tk.id < 0) break;
         const int len = tk.len;
         unsigned char* rec = tk.rec;
-        if (tid < C) s_beta[tid] = tid < len ? to_f32(beta[(tk.c0 + tid) * H + tk.h]) : 0.f;
+        const float* s_beta = s_beta2 + 64 * (it & 1);
         failed = !mbar_wait(bar_tma, it & 1, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
 
@@ -357,6 +397,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (qr == 2) { x_gm[c] = g[0]; x_egm[c] = expf(g[0]); }     // row 32
             if (qr == 3) { x_gc[c] = g[15]; x_gam[c] = expf(g[15]); }   // row 63 (padded rows add nothing)
         }
+        if (tid == 0) bulk_wait_read();  // the previous record has left the Mt and Qh staging tiles
         __syncthreads();
         {
             const float gm = x_gm[c], gC = x_gc[c], egm = x_egm[c];
@@ -426,6 +467,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mma_tf32_ts(tmem + TM_D1, tmem + TM_A1 + 8 * kk, bkm + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4),
                             id1, kk > 0);
             mma_commit(bar_mma);
+            slots[aft] = walker.next();  // while the tensor cores run: the task after the next
         }
         failed = !mbar_wait(bar_mma, 0, kWaitPolls);  // bar_mma completes twice per task: parities 0, 1
         if (__syncthreads_or(failed)) { failed = true; break; }
@@ -528,7 +570,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int kk = 0; kk < C / 8; ++kk)
                 mma_tf32(tmem + TM_PW, dp + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), bw + static_cast<uint64_t>(kk) * 64,
                          id_pw, kk > 0);
-            mma_commit(bar_pw);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk) {
                 const uint64_t kt = dkt + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
@@ -540,16 +581,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             mma_commit(bar_rest);
         }
-        failed = !mbar_wait(bar_pw, it & 1, kWaitPolls);
+        failed = !mbar_wait(bar_rest, it & 1, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        {   // Qh = Q e^G - P W (row t = 16 q4 + lane, channels 32 qr ..) -> record, MN-major
+        {   // Qh = Q e^G - P W (row t = 16 q4 + lane, channels 32 qr ..) -> staging, K-major rows t
             const int t = 16 * q4 + lane;
             const bool live = t < len;
             float x[32];
             tmem_ld32(tq + TM_PW + 32 * qr, x);
             if (lane < 16) {
-                float* gq = reinterpret_cast<float*>(rec + wy::REC_Q);
+                unsigned char* row = sm + STG_Q + qr * 8192 + t * 128;  // K-block qr, row t
 #pragma unroll
                 for (int e8 = 0; e8 < 4; ++e8) {
                     const int cc = 32 * qr + 8 * e8;
@@ -558,38 +599,35 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const float4 e0 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc, 64));
                     const float4 e1 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc + 4, 64));
                     const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                    float qh[8];
 #pragma unroll
                     for (int w = 0; w < 8; ++w)
-                        gq[sw32b_off(cc + w, t, 128) >> 2] =
-                            to_tf32((live ? qv[w] * ev[w] * x_egm[cc + w] : 0.f) - x[8 * e8 + w]);
+                        qh[w] = to_tf32((live ? qv[w] * ev[w] * x_egm[cc + w] : 0.f) - x[8 * e8 + w]);
+                    *reinterpret_cast<float4*>(row + (((2 * e8) ^ (t & 7)) << 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
+                    *reinterpret_cast<float4*>(row + (((2 * e8 + 1) ^ (t & 7)) << 4)) =
+                        make_float4(qh[4], qh[5], qh[6], qh[7]);
                 }
             }
         }
-        __syncthreads();  // the staging buffers are free: bring in the next task's tiles
-        if (tid == 0) {
-            const Task tn = slots[(it + 1) & 1];
-            Task ta;
-            ta.id = -1;
-            if (tn.id >= 0) {
-                issue_loads(tn, false);
-                ++loads_issued;
-                ta = next_task(tn.id + gridDim.x, gridDim.x, ntasks, cu_seqlens, T_total, N, H, ws, flags);
-                if (ta.id >= 0) issue_loads(ta, true);
-            }
-            slots[it & 1] = ta;  // this task's slot now holds the one after next
+        const Task tn = slots[nxt];
+        if (tid == 0 && tn.id >= 0) {
+            mbar_arrive_expect_tx(bar_tma, kStageBytes);
+            ++loads_issued;
         }
-        failed = !mbar_wait(bar_rest, it & 1, kWaitPolls);
-        if (__syncthreads_or(failed)) { failed = true; break; }
-        tc_fence_after_sync();
-        {   // Mt = Diag(e^{g_C}) - Kt^T W (row i = c, columns j = 32 qr ..) -> record, MN-major
+        __syncthreads();  // q and E are read: the next task's tiles may come into the staging buffers
+        if (lane == 0 && warp < kLoads && tn.id >= 0) load_box(tn, warp);
+        load_beta(tn, (it + 1) & 1);
+        {   // Mt = Diag(e^{g_C}) - Kt^T W (row i = c, columns j = 32 qr ..) -> staging, K-major rows i
             float x[32];
             tmem_ld32(tq + TM_KW + 32 * qr, x);
             const float gam = x_gam[c];
-            float* gm_ = reinterpret_cast<float*>(rec + wy::REC_M);
+            unsigned char* row = sm + STG_M + qr * 16384 + c * 128;  // K-block qr, row i
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int j = 32 * qr + e;
-                gm_[sw32b_off(j, c, 128) >> 2] = to_tf32((c == j ? gam : 0.f) - x[e]);
+            for (int e4 = 0; e4 < 8; ++e4) {
+                float m[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) m[u] = to_tf32((c == 32 * qr + 4 * e4 + u ? gam : 0.f) - x[4 * e4 + u]);
+                *reinterpret_cast<float4*>(row + ((e4 ^ (c & 7)) << 4)) = make_float4(m[0], m[1], m[2], m[3]);
             }
         }
         {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record
@@ -606,8 +644,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int s4 = 0; s4 < 4; ++s4)
                 gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4], y[4 * s4 + 1], y[4 * s4 + 2], y[4 * s4 + 3]);
         }
+        fence_async_smem();
         tc_fence_before_sync();
         __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) bulk_store(rec + wy::REC_M + b * 16384, sm + STG_M + b * 16384, 16384);
+            bulk_store(rec + wy::REC_Q, sm + STG_Q, 16384);
+            bulk_store(rec + wy::REC_Q + 16384, sm + STG_Q + 16384, 16384);
+            bulk_commit();
+        }
     }
 
     if (failed && tid == 0) {
@@ -615,6 +661,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (loads_issued > 0) mbar_wait(bar_tma, (loads_issued - 1) & 1, kWaitPolls);
         raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
     }
+    if (tid == 0) bulk_wait_read();  // the bulk stores read shared memory until they complete
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {

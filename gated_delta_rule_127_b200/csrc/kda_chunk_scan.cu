@@ -13,7 +13,8 @@
 // state is read by the tensor cores as tf32 (its low 13 mantissa bits ignored) and accumulated in
 // fp32; it is stored in fp32 at the end.
 //
-// Roles (320 threads): warps 0-7 fill the accumulators and store o and the final state -- warp w
+// Roles (320 threads): warps 0-7 fill the accumulators and write o (through a shared-memory tile and
+// one TMA store per full chunk) and the final state -- warp w
 // serves value columns dv = 32 (w % 4) .. +31 (its tensor-memory lanes) and half w / 4 of the
 // accumulator columns, and holds the next chunk's share of B and Uo in registers while the current
 // chunk's MMAs run; warp 8 lane 0 brings each chunk's Mt and Qh operand tiles into a two-stage
@@ -26,6 +27,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_sm100.cuh"
+#include "kda_tma.h"
 #include "kda_wy.cuh"
 
 namespace kda {
@@ -45,7 +47,8 @@ constexpr uint32_t kWaitPolls = 1u << 26;
 constexpr uint32_t STAGE_BYTES = 98304;  // Mt tile (64 KB) + Qh tile (32 KB)
 constexpr uint32_t OFF_STAGE0 = 0;
 constexpr uint32_t OFF_STAGE1 = STAGE_BYTES;
-constexpr uint32_t OFF_BARS = 2 * STAGE_BYTES;  // full[2], empty[2], chain, sinit[2], odone[2]
+constexpr uint32_t OFF_OST = 2 * STAGE_BYTES;   // o tile of one chunk, [64][128] in dtype_o (32 KB max)
+constexpr uint32_t OFF_BARS = OFF_OST + 32768;  // full[2], empty[2], chain, sinit[2], odone[2]
 constexpr uint32_t OFF_SLOT = OFF_BARS + 9 * 8;
 constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
@@ -79,8 +82,18 @@ __device__ __forceinline__ void store_o(void* o, int64_t idx, float x, bool f32)
     else static_cast<__nv_bfloat16*>(o)[idx] = __float2bfloat16_rn(x);
 }
 
+__device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(tmap),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __global__ void __launch_bounds__(THREADS, 1)
-chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_state,
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char* __restrict__ ws,
+                  const float* initial_state,
                   const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H, void* __restrict__ o_ptr,
                   int o_is_f32, float* final_state, unsigned int* flags) {
     extern __shared__ unsigned char smem_raw[];
@@ -139,15 +152,33 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
             }
             tmem_st_wait();
         }
-        auto emit_o = [&](int c) {  // tokens 32 g .. 32 g + 31 of O_c^T (output buffer c & 1) -> o
+        auto emit_o = [&](int c, const float (&x)[32]) {  // tokens 32 g .. 32 g + 31 of O_c -> o
             const int64_t c0 = t0 + static_cast<int64_t>(c) * C;
             const int len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
-            float x[32];
-            tmem_ld32(tq + TM_O + 64 * (c & 1) + 32 * g, x);
+            if (len == C) {  // whole chunk: rows into the o tile, then one TMA store
+                if (tid == 0) bulk_wait_read();  // the previous tile has left shared memory
+                group_sync(1, DATA_THREADS);
+                if (o_is_f32) {
+                    float* ost = reinterpret_cast<float*>(sm + OFF_OST);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int t = 32 * g + e;
-                if (t < len) store_o(o_ptr, ((c0 + t) * H + h) * DV + dv, x[e], o_is_f32 != 0);
+                    for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DV + dv] = x[e];
+                } else {
+                    __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OFF_OST);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DV + dv] = __float2bfloat16_rn(x[e]);
+                }
+                fence_async_smem();
+                group_sync(1, DATA_THREADS);
+                if (tid == 0) {
+                    tma_store_3d(&tm_o, sm + OFF_OST, 0, h, static_cast<int>(c0));
+                    bulk_commit();
+                }
+            } else {  // the sequence's last, partial chunk: its own rows only
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int t = 32 * g + e;
+                    if (t < len) store_o(o_ptr, ((c0 + t) * H + h) * DV + dv, x[e], o_is_f32 != 0);
+                }
             }
         };
         // this thread's share of chunk c's B^T (rows i = 64 g .. +63) and Uo^T (tokens 32 g .. +31)
@@ -173,11 +204,14 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
         bool ok = true;
         if (nc > 0) fetch(0);
         for (int c = 0; c < nc && ok; ++c) {
+            // O_{c-2} out of output buffer c & 1 first, so chunk c's accumulators can be signalled before
+            // O_{c-2} is written to memory
+            float ox[32];
             if (c >= 2) {
                 ok = wait_or_abort(odone + (c & 1), ((c - 2) >> 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after_sync();
-                emit_o(c - 2);
+                tmem_ld32(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
             }
             const uint32_t sb = TM_S + 128 * ((c + 1) % 3) + 64 * g;
             put32(tq + sb, pb);
@@ -187,12 +221,15 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
             tc_fence_before_sync();
             mbar_arrive(sinit + (c & 1));
             if (c + 1 < nc) fetch(c + 1);
+            if (c >= 2) emit_o(c - 2, ox);
         }
         for (int c = nc - 2 < 0 ? 0 : nc - 2; c < nc && ok; ++c) {
             ok = wait_or_abort(odone + (c & 1), (c >> 1) & 1, abort);
             if (!ok) break;
             tc_fence_after_sync();
-            emit_o(c);
+            float ox[32];
+            tmem_ld32(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
+            emit_o(c, ox);
         }
         if (ok && final_state) {  // after the last output MMA, the last state MMA is complete too
             const uint32_t sb = TM_S + 128 * (nc % 3);
@@ -237,8 +274,8 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t sbase = smem_u32(sm);
-            constexpr uint32_t id_s = idesc_tf32(128, 128, false, true);
-            constexpr uint32_t id_o = idesc_tf32(128, 64, false, true);
+            constexpr uint32_t id_s = idesc_tf32(128, 128, false, false);
+            constexpr uint32_t id_o = idesc_tf32(128, 64, false, false);
             int committed = 0;
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
@@ -247,18 +284,18 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
                 if (c >= 1 && !wait_or_abort(chain, (c - 1) & 1, abort)) break;
                 tc_fence_after_sync();
                 const uint32_t st = sbase + (s ? OFF_STAGE1 : OFF_STAGE0);
-                const uint64_t bm = sw128b32_desc(st, 128 * 128, 512);           // Mt, MN-major
-                const uint64_t bq = sw128b32_desc(st + 65536, 128 * 128, 512);   // Qh, MN-major
+                const uint64_t bm = sw128_desc(st, 16, 1024);          // Mt, K-major rows i
+                const uint64_t bq = sw128_desc(st + 65536, 16, 1024);  // Qh, K-major rows t
                 const uint32_t a_s = tmem + TM_S + 128 * (c % 3);
                 const uint32_t d_s = tmem + TM_S + 128 * ((c + 1) % 3);
                 const uint32_t d_o = tmem + TM_O + 64 * s;
 #pragma unroll
-                for (int kk = 0; kk < DK / 8; ++kk)  // K-step: 8 K-rows of 128 bytes
-                    mma_tf32_ts(d_s, a_s + 8 * kk, bm + static_cast<uint64_t>(kk) * 64, id_s, 1);
+                for (int kk = 0; kk < DK / 8; ++kk)  // K-step: 32 bytes within a 128-byte K-block
+                    mma_tf32_ts(d_s, a_s + 8 * kk, bm + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), id_s, 1);
                 mma_commit(chain);
 #pragma unroll
                 for (int kk = 0; kk < DK / 8; ++kk)
-                    mma_tf32_ts(d_o, a_s + 8 * kk, bq + static_cast<uint64_t>(kk) * 64, id_o, 1);
+                    mma_tf32_ts(d_o, a_s + 8 * kk, bq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_o, 1);
                 mma_commit(empty + s);
                 mma_commit(odone + s);
                 committed = c + 1;
@@ -269,6 +306,7 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
         __syncwarp();
     }
 
+    if (tid == 0) bulk_wait_all();  // o tiles written before the CTA's shared memory goes away
     __syncthreads();
     if (tid == 0 && *abort) raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
     tc_fence_before_sync();
@@ -282,12 +320,18 @@ chunk_scan_kernel(const unsigned char* __restrict__ ws, const float* initial_sta
 }  // namespace
 
 cudaError_t launch_chunk_scan(const ChunkArgs& a) {
+    CUtensorMap mo;
+    const bool f32 = a.dtype_o == KDA_FP32;
+    if (!tma_encode_thd(&mo, a.o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2,
+                        DV, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T_total), DV, C,
+                        CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
     cudaError_t err =
         cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int64_t blocks = static_cast<int64_t>(a.N) * a.H;
     chunk_scan_kernel<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
-        static_cast<const unsigned char*>(a.workspace), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
+        mo, static_cast<const unsigned char*>(a.workspace), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
         a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags);
     return cudaGetLastError();
 }

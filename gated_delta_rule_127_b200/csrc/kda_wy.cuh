@@ -11,11 +11,11 @@
 // computed in parallel; the scan then needs one dk x dk x dv and one C x dk x dv product per chunk.
 //
 // Record of one (chunk, head), REC_BYTES bytes, fp32:
-//   REC_M  Mt as the scan's B operand (K = key channel j, N = key channel i), MN-major in the 128-byte
-//          layout with 32-byte atoms: four 32-channel N-blocks of 128 K-rows x 128 bytes; element (i, j)
-//          at sw32b_off(j, i, 128).  Rounded to tf32.
-//   REC_Q  Qh as the scan's B operand (K = j, N = token t): two 32-token N-blocks of 128 K-rows x 128
-//          bytes; element (t, j) at sw32b_off(j, t, 128).  Rounded to tf32.
+//   REC_M  Mt as the scan's B operand (K = key channel j, N = key channel i), K-major with the 128-byte
+//          swizzle: four 32-channel K-blocks of 128 rows x 128 bytes; element (i, j) at
+//          sw128_off(i, j, 128).  Rounded to tf32.
+//   REC_Q  Qh as the scan's B operand (K = j, N = token t): four K-blocks of 64 rows x 128 bytes;
+//          element (t, j) at sw128_off(t, j, 64).  Rounded to tf32.
 //   REC_B  B transposed and interleaved by four: element (i, dv) at float index (i / 4) * 512 + dv * 4
 //          + i % 4, so thread dv reading float4 number (i / 4) * 128 + dv gets B[i..i+3][dv] and a
 //          warp's read, like the writer's store of four rows, is one contiguous 512-byte run.
