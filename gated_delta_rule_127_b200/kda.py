@@ -43,6 +43,9 @@ def load_library() -> ctypes.CDLL:
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, i32, i32, i32,
                                   vp, vp, vp, sz, vp]
     lib.kda_chunk_fwd.restype = i32
+    lib.kda_chunk_fwd_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, i32,
+                                                 i32, i32, vp, vp, vp]
+    lib.kda_chunk_fwd_static_scratch.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
     lib.kda_decode_step.restype = i32
     lib.kda_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -164,6 +167,56 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: 
                                _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd")
+    return o, final_state
+
+
+def kda_chunk_fwd_static_scratch(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                                 beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
+                                 cu_seqlens: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
+                                 chunk_size: int = 64, o: Optional[torch.Tensor] = None,
+                                 final_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
+                                 dtype_o: Optional[torch.dtype] = None,
+                                 stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kda_chunk_fwd_static_scratch (include/kda.h): kda_chunk_fwd with the library's fixed scratch
+    instead of a workspace.  Same arguments and results as kda_chunk_fwd."""
+    lib = load_library()
+    if q.dim() != 3 or k.shape != q.shape or log_alpha.shape != q.shape or v.dim() != 3 or beta.dim() != 2:
+        raise ValueError("expected q, k, log_alpha [T, H, dk], v [T, H, dv], beta [T, H]")
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if v.shape[:2] != (T, H) or beta.shape != (T, H):
+        raise ValueError("v / beta shapes do not match q")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor")
+        N = cu_seqlens.shape[0] - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k, v must share a dtype")
+    if log_alpha.dtype != beta.dtype:
+        raise TypeError("log_alpha and beta must share a dtype")
+    device = q.device
+    if dtype_o is None:
+        dtype_o = o.dtype if o is not None else q.dtype
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=dtype_o, device=device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=device)
+    if initial_state is not None and (initial_state.dtype != torch.float32 or initial_state.shape != (N, H, dk, dv)):
+        raise ValueError("initial_state must be fp32 [N, H, dk, dv]")
+    if final_state is not None and (final_state.dtype != torch.float32 or final_state.shape != (N, H, dk, dv)):
+        raise ValueError("final_state must be fp32 [N, H, dk, dv]")
+    _check_cuda(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, initial_state=initial_state,
+                     cu_seqlens=cu_seqlens, o=o, final_state=final_state), device)
+    with torch.cuda.device(device):
+        st = lib.kda_chunk_fwd_static_scratch(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                              _ptr(initial_state), _ptr(cu_seqlens), T, N, H, dk, dv, chunk_size,
+                                              _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"),
+                                              _dtype_code(o, "o"), _ptr(o), _ptr(final_state),
+                                              _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_static_scratch")
     return o, final_state
 
 

@@ -109,6 +109,34 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          void* o, float* final_state,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of the device array kda_chunk_fwd_static_scratch works in (32 MiB). */
+#define KDA_STATIC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * kda_chunk_fwd for callers that cannot allocate device memory: the same arguments without the
+ * workspace, the same results (the same kernels run).  The pages have no counterpart to this entry
+ * point; it only changes where the scratch lives.  It allocates nothing: its scratch is a
+ * file-scope device array of KDA_STATIC_SCRATCH_BYTES, reserved on a device when the library's
+ * device code is loaded there, whose address is looked up once per device on the first call made
+ * with that device current.
+ *   - Limit: calls whose kda_chunk_fwd_workspace_size(...) exceeds KDA_STATIC_SCRATCH_BYTES return
+ *     KDA_ERR_UNSUPPORTED before any CUDA call.  32 MiB holds 170 chunk records, one per 64-token
+ *     chunk slot and head (slots = T_total / 64 + N + 1); e.g. 2 sequences x 2048 tokens x 2 heads
+ *     uses 134.  Calls that need no workspace (fp32 q/k/v, dk or dv = 64) have no limit.
+ *   - Nothing in the scratch has to start at zero: every part a call reads is written earlier in the
+ *     same call.
+ *   - Every call on a device shares the one array: two calls that can run at the same time (on
+ *     different streams, or from host threads without ordering between them) race on it and corrupt
+ *     each other's results.  Order such calls (one stream, or synchronise in between).
+ * Other statuses and behaviour as kda_chunk_fwd.
+ */
+KDA_API kda_status kda_chunk_fwd_static_scratch(const void* q, const void* k, const void* v,
+                         const void* log_alpha, const void* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
+                         void* o, float* final_state, void* stream);
+
 /*
  * One recurrent decode step for B sequences (one new token each), state updated in place.
  *

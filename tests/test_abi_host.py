@@ -99,3 +99,11 @@ def test_workspace_size_is_a_pure_host_function(lib):
     # one 192 KB record per (chunk slot, head); slots = T / 64 + N + 1
     assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) == (512 + 2) * 32 * 196608
     assert kda.kda_chunk_fwd_workspace_size(1000, 3, 2, 128, 128) == (15 + 4) * 2 * 196608
+
+
+def test_static_scratch_rejects_oversize_before_any_cuda_call(lib):
+    # 65536 tokens x 4 heads needs (1024 + 2) x 4 chunk records: more than the 32 MiB array holds
+    assert kda.kda_chunk_fwd_workspace_size(65536, 1, 4, 128, 128) > 32 << 20
+    st = lib.kda_chunk_fwd_static_scratch(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 65536, 1, 4, 128, 128, 64,
+                                          kda.KDA_BF16, kda.KDA_FP32, kda.KDA_FP32, FAKE, None, None)
+    assert st == kda.KDA_ERR_UNSUPPORTED
