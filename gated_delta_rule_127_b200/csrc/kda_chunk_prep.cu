@@ -46,7 +46,7 @@ using wy::DK;
 using wy::DV;
 
 constexpr int THREADS = 512;
-constexpr int TP = 64;  // row stride (floats) of the fp32 A and T tiles
+constexpr int TP = 68;  // row stride (floats) of the fp32 A and T tiles (conflict-free MMA fragment reads)
 constexpr float kAnchorLimit = 80.f;
 constexpr uint32_t kWaitPolls = 1u << 26;
 
@@ -68,9 +68,9 @@ constexpr uint32_t SMEM_USED = 221832;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 // after MMA 1 (k, v staging and K- are dead):
 constexpr uint32_t OFF_A = 49152;      // A fp32 [64][TP]
-constexpr uint32_t OFF_T32 = 65536;    // T fp32 [64][TP]
-constexpr uint32_t OFF_TIMG = 81920;   // T K-major rows r x K s (64), MMA 2's A
-constexpr uint32_t OFF_P = 98304;      // P K-major rows t x K s (64), A of MMA 3 and B of MMA 6
+constexpr uint32_t OFF_T32 = 66560;    // T fp32 [64][TP]
+constexpr uint32_t OFF_TIMG = 49152;   // T K-major rows r x K s (64), MMA 2's A (over A, once T is formed)
+constexpr uint32_t OFF_P = 84992;      // P K-major rows t x K s (64), A of MMA 3 and B of MMA 6
 // record staging once MMAs 3-6 are done, outside the input staging so the next task's tiles can load:
 constexpr uint32_t STG_M = OFF_B8;     // Mt K-major rows i x K j (128), 64 KB
 constexpr uint32_t STG_Q = OFF_KT;     // Qh K-major rows t x K j (128), 32 KB
@@ -179,9 +179,42 @@ struct TaskWalker {
     }
 };
 
+// One 16 x 8 tile of X Y on the warp's tensor cores (mma.sync m16n8k8, tf32 operands rounded to
+// nearest, fp32 accumulation): X row-major with row stride xs (the tile's 16 rows, K = kn columns), Y
+// row-major with row stride ys (K = kn rows, the tile's 8 columns).  Fragment layout of the m16n8k8
+// tf32 shape: lane = 4 g + t holds X[g][t], X[g+8][t], X[g][t+4], X[g+8][t+4] and Y[t][g], Y[t+4][g],
+// and receives D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1].
+__device__ __forceinline__ void warp_tile_16x8(const float* x, int xs, const float* y, int ys, int kn, float (&d)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    d[0] = d[1] = d[2] = d[3] = 0.f;
+    for (int k0 = 0; k0 < kn; k0 += 8) {
+        const uint32_t a0 = __float_as_uint(to_tf32(x[g * xs + k0 + t]));
+        const uint32_t a1 = __float_as_uint(to_tf32(x[(g + 8) * xs + k0 + t]));
+        const uint32_t a2 = __float_as_uint(to_tf32(x[g * xs + k0 + t + 4]));
+        const uint32_t a3 = __float_as_uint(to_tf32(x[(g + 8) * xs + k0 + t + 4]));
+        const uint32_t b0 = __float_as_uint(to_tf32(y[(k0 + t) * ys + g]));
+        const uint32_t b1 = __float_as_uint(to_tf32(y[(k0 + t + 4) * ys + g]));
+        asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+// Stores the negated tile at z (row stride zs) or, with neg = false, the tile itself.
+__device__ __forceinline__ void warp_store_16x8(float* z, int zs, const float (&d)[4], bool neg) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const float sg = neg ? -1.f : 1.f;
+    z[g * zs + 2 * t] = sg * d[0];
+    z[g * zs + 2 * t + 1] = sg * d[1];
+    z[(g + 8) * zs + 2 * t] = sg * d[2];
+    z[(g + 8) * zs + 2 * t + 1] = sg * d[3];
+}
+
 // T = (I + A)^{-1} for A strictly lower (fp32, row stride TP) into tm, fully written (zero above the
-// diagonal).  xs: 1024 floats of scratch.  The 16 x 16 diagonal blocks by forward substitution, then
-// two merges of [[T1, 0], [T21, T2]] with T21 = -T2 A21 T1: 16 -> 32 (both halves at once) and 32 -> 64.
+// diagonal).  xs: 1024 floats of scratch.  The 16 x 16 diagonal blocks by forward substitution in fp32,
+// then two merges of [[T1, 0], [T21, T2]] with T21 = -T2 A21 T1: 16 -> 32 (both halves at once) and
+// 32 -> 64, whose products run as 16 x 8 tiles on the warps' tensor cores with tf32 operands (these
+// blocks reach the rest of the chunk only through tf32 products; an fp64 emulation against the
+// oracle shows no loss from it).
 __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, float* xs) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (warp < 4) {
@@ -216,61 +249,30 @@ __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, f
         }
     }
     __syncthreads();
-    {   // 16 -> 32, blocks p = 0, 1 (rows 32 p .. 32 p + 31): X = A_{2p+1,2p} T_{2p,2p}
-        const int p = tid >> 8, r = (tid >> 4) & 15, cc = tid & 15;
-        const float* arow = am + (32 * p + 16 + r) * TP + 32 * p;
-        const float* tcol = tm + (32 * p) * TP + 32 * p + cc;
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; m += 4) {
-            const float4 a = *reinterpret_cast<const float4*>(arow + m);
-            a0 += a.x * tcol[m * TP] + a.y * tcol[(m + 1) * TP];
-            a1 += a.z * tcol[(m + 2) * TP] + a.w * tcol[(m + 3) * TP];
-        }
-        xs[tid] = a0 + a1;
-        __syncthreads();
-        //                                           T_{2p+1,2p} = -T_{2p+1,2p+1} X
-        const float* trow = tm + (32 * p + 16 + r) * TP + 32 * p + 16;
-        const float* xcol = xs + p * 256 + cc;
-        float b0 = 0.f, b1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; m += 4) {
-            const float4 t = *reinterpret_cast<const float4*>(trow + m);
-            b0 += t.x * xcol[m * 16] + t.y * xcol[(m + 1) * 16];
-            b1 += t.z * xcol[(m + 2) * 16] + t.w * xcol[(m + 3) * 16];
-        }
-        tm[(32 * p + 16 + r) * TP + 32 * p + cc] = -(b0 + b1);
+    const int p = warp >> 1, nt = warp & 1;  // 16 -> 32: warps 0..3, block pair p, 8-column tile nt
+    if (warp < 4) {  // X_p = A_{2p+1,2p} T_{2p,2p}
+        float d[4];
+        warp_tile_16x8(am + (32 * p + 16) * TP + 32 * p, TP, tm + (32 * p) * TP + 32 * p + 8 * nt, TP, 16, d);
+        warp_store_16x8(xs + p * 256 + 8 * nt, 16, d, false);
     }
     __syncthreads();
-    // 32 -> 64: X = A21 T1 (rows 32..63, columns 0..31), then T21 = -T2 X; two elements per thread
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int e = tid + THREADS * u, r = e >> 5, cc = e & 31;
-        const float* arow = am + (32 + r) * TP;
-        const float* tcol = tm + cc;
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 32; m += 4) {
-            const float4 a = *reinterpret_cast<const float4*>(arow + m);
-            a0 += a.x * tcol[m * TP] + a.y * tcol[(m + 1) * TP];
-            a1 += a.z * tcol[(m + 2) * TP] + a.w * tcol[(m + 3) * TP];
-        }
-        xs[e] = a0 + a1;
+    if (warp < 4) {  // T_{2p+1,2p} = -T_{2p+1,2p+1} X_p
+        float d[4];
+        warp_tile_16x8(tm + (32 * p + 16) * TP + 32 * p + 16, TP, xs + p * 256 + 8 * nt, 16, 16, d);
+        warp_store_16x8(tm + (32 * p + 16) * TP + 32 * p + 8 * nt, TP, d, true);
     }
     __syncthreads();
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int e = tid + THREADS * u, r = e >> 5, cc = e & 31;
-        const float* trow = tm + (32 + r) * TP + 32;
-        const float* xcol = xs + cc;
-        float b0 = 0.f, b1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 32; m += 4) {
-            const float4 t = *reinterpret_cast<const float4*>(trow + m);
-            b0 += t.x * xcol[m * 32] + t.y * xcol[(m + 1) * 32];
-            b1 += t.z * xcol[(m + 2) * 32] + t.w * xcol[(m + 3) * 32];
-        }
-        tm[(32 + r) * TP + cc] = -(b0 + b1);
+    const int mt = warp >> 2, ct = warp & 3;  // 32 -> 64: warps 0..7, 16-row tile mt, 8-column tile ct
+    if (warp < 8) {  // X = A21 T1
+        float d[4];
+        warp_tile_16x8(am + (32 + 16 * mt) * TP, TP, tm + 8 * ct, TP, 32, d);
+        warp_store_16x8(xs + (16 * mt) * 32 + 8 * ct, 32, d, false);
+    }
+    __syncthreads();
+    if (warp < 8) {  // T21 = -T2 X
+        float d[4];
+        warp_tile_16x8(tm + (32 + 16 * mt) * TP + 32, TP, xs + 8 * ct, 32, 32, d);
+        warp_store_16x8(tm + (32 + 16 * mt) * TP + 8 * ct, TP, d, true);
     }
     __syncthreads();
 }
@@ -304,26 +306,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     constexpr uint32_t kGateBytes = C * DK * sizeof(TG);
     constexpr uint32_t kStageBytes = 3 * C * DK * 2 + kGateBytes;
-    // Box j of the task's q, k, v and log_alpha tiles into the staging buffers (completion on bar_tma,
-    // whose expected byte count kStageBytes is set once per task).  The boxes are issued by different
-    // warps so that no thread serialises all of them.
-    constexpr int kLoads = sizeof(TG) == 4 ? 10 : 8;
+    // Tile j (k, q, v, log_alpha) of a task into the staging buffers: one box covering all of the
+    // tile's 128-byte column blocks (completion on bar_tma, whose expected byte count kStageBytes is
+    // set once per task).  The four are issued by different warps.
+    constexpr int kLoads = 4;
     auto load_box = [&](const Task& t, int j) {
-        const int y = static_cast<int>(t.c0), hh = t.h;
-        const CUtensorMap* m = j < 2 ? &tm_k : j < 4 ? &tm_q : j < 6 ? &tm_v : &tm_g;
-        uint32_t dst;
-        int x;
-        if (j < 6) {
-            dst = (j < 2 ? OFF_SK : j < 4 ? OFF_SQ : OFF_SV) + 8192 * (j & 1);
-            x = 64 * (j & 1);
-        } else if (sizeof(TG) == 4) {
-            dst = OFF_G + 8192 * (j - 6);
-            x = 32 * (j - 6);
-        } else {
-            dst = OFF_G + 16384 + 8192 * (j - 6);
-            x = 64 * (j - 6);
-        }
-        tma_load_3d(sm + dst, m, x, hh, y, bar_tma);
+        const CUtensorMap* m = j == 0 ? &tm_k : j == 1 ? &tm_q : j == 2 ? &tm_v : &tm_g;
+        const uint32_t dst = j == 0 ? OFF_SK : j == 1 ? OFF_SQ : j == 2 ? OFF_SV : OFF_G + (sizeof(TG) == 4 ? 0u : 16384u);
+        tma_load_4d(sm + dst, m, 0, static_cast<int>(t.c0), 0, t.h, bar_tma);
     };
 
     uint32_t loads_issued = 0;  // thread 0: staging loads issued (bar_tma phases)
@@ -683,11 +673,13 @@ cudaError_t launch_prep(const ChunkArgs& a) {
     const uint64_t T = static_cast<uint64_t>(a.T_total), H = static_cast<uint64_t>(a.H);
     const CUtensorMapDataType gdt =
         sizeof(TG) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const uint32_t gbox = sizeof(TG) == 4 ? 32 : 64;  // 128 bytes of channels per box
-    if (!tma_encode_thd(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, H, T, 64, C, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !tma_encode_thd(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, H, T, 64, C, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !tma_encode_thd(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, H, T, 64, C, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !tma_encode_thd(&mg, a.log_alpha, gdt, sizeof(TG), DK, H, T, gbox, C, CU_TENSOR_MAP_SWIZZLE_128B))
+    const uint32_t gblk = sizeof(TG) == 4 ? 32 : 64;  // 128 bytes of channels per column block
+    constexpr CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    constexpr CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!tma_encode_blocks(&mq, a.q, bf, 2, DK, H, T, 64, C, sw) ||
+        !tma_encode_blocks(&mk, a.k, bf, 2, DK, H, T, 64, C, sw) ||
+        !tma_encode_blocks(&mv, a.v, bf, 2, DV, H, T, 64, C, sw) ||
+        !tma_encode_blocks(&mg, a.log_alpha, gdt, sizeof(TG), DK, H, T, gblk, C, sw))
         return cudaErrorInvalidValue;
     auto kern = chunk_prep_kernel<TG>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);

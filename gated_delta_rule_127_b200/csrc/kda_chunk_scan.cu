@@ -1,5 +1,6 @@
 // kda_chunk_scan.cu -- the inter-chunk half of the chunked KDA prefill on the sm_100a tensor cores:
-// per (sequence, head), walk the chunks in order carrying the fp32 state in tensor memory.
+// per (sequence, head, half of the value columns), walk the chunks in order carrying the fp32 state in
+// tensor memory.
 //
 // "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "청크 단위 병렬 알고리듬": each chunk
 // starts from the previous chunk's final state.  With the chunk record of kda_wy.cuh (computed for
@@ -7,17 +8,20 @@
 //   S_{n+1} = Mt_n S_n + B_n,      O_n = Qh_n S_n + Uo_n,
 // which the CTA runs transposed, so the state is the tensor cores' A operand straight from tensor
 // memory and each chunk's result is the next chunk's operand without passing through registers:
-//   S_{n+1}^T = B_n^T + S_n^T Mt_n^T    (M = dv = 128, N = 128, K = dk = 128: 16 MMAs)
-//   O_n^T     = Uo_n^T + S_n^T Qh_n^T   (M = 128, N = 64, K = 128: 16 MMAs)
+//   S_{n+1}^T = B_n^T + S_n^T Mt_n^T    (M = 64 value columns, N = 128, K = dk = 128: 16 MMAs)
+//   O_n^T     = Uo_n^T + S_n^T Qh_n^T   (M = 64, N = 64, K = 128: 16 MMAs)
+// Value columns are independent in the recurrence, so each head is split between two CTAs by value
+// columns: an M = 64 MMA takes the tensor cores as long as an M = 128 one at these widths, and the
+// split halves each CTA's share of the B and Uo stream while both read the same Mt and Qh tiles.
 // The accumulators start from B_n^T and Uo_n^T, written into tensor memory by the data warps.  The
 // state is read by the tensor cores as tf32 (its low 13 mantissa bits ignored) and accumulated in
 // fp32; it is stored in fp32 at the end.
 //
 // Roles (320 threads): warps 0-7 fill the accumulators and write o (through a shared-memory tile and
-// one TMA store per full chunk) and the final state -- warp w
-// serves value columns dv = 32 (w % 4) .. +31 (its tensor-memory lanes) and half w / 4 of the
-// accumulator columns, and holds the next chunk's share of B and Uo in registers while the current
-// chunk's MMAs run; warp 8 lane 0 brings each chunk's Mt and Qh operand tiles into a two-stage
+// one TMA store per full chunk) and the final state -- lanes 0..15 of warp w serve the value columns
+// 16 (w % 4) .. +15 of the CTA's half (the M = 64 accumulator rows, tensor-memory lanes 32 (w % 4) ..
+// +15) and half w / 4 of the accumulator columns, and hold the next chunk's share of B and Uo in
+// registers while the current chunk's MMAs run; warp 8 lane 0 brings each chunk's Mt and Qh operand tiles into a two-stage
 // shared-memory ring with bulk copies (and asks L2 for the B and Uo of the chunk after); warp 9
 // lane 0 issues the MMAs.
 // Tensor memory: three state buffers (S_n read while S_{n+1} accumulates and S_{n+2}'s B is written)
@@ -44,11 +48,12 @@ constexpr int LOADER_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr uint32_t kWaitPolls = 1u << 26;
 
+constexpr int DVH = 64;                  // value columns per CTA
 constexpr uint32_t STAGE_BYTES = 98304;  // Mt tile (64 KB) + Qh tile (32 KB)
 constexpr uint32_t OFF_STAGE0 = 0;
 constexpr uint32_t OFF_STAGE1 = STAGE_BYTES;
-constexpr uint32_t OFF_OST = 2 * STAGE_BYTES;   // o tile of one chunk, [64][128] in dtype_o (32 KB max)
-constexpr uint32_t OFF_BARS = OFF_OST + 32768;  // full[2], empty[2], chain, sinit[2], odone[2]
+constexpr uint32_t OFF_OST = 2 * STAGE_BYTES;   // o tile of one chunk, [64][64] in dtype_o (16 KB max)
+constexpr uint32_t OFF_BARS = OFF_OST + 16384;  // full[2], empty[2], chain, sinit[2], odone[2]
 constexpr uint32_t OFF_SLOT = OFF_BARS + 9 * 8;
 constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
@@ -109,8 +114,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
     volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = static_cast<int>(blockIdx.x % H);
-    const int n = static_cast<int>(blockIdx.x / H);
+    const int half = static_cast<int>(blockIdx.x & 1);  // value columns 64 half .. +63
+    const int h = static_cast<int>((blockIdx.x >> 1) % H);
+    const int n = static_cast<int>((blockIdx.x >> 1) / H);
     int64_t t0, t1;
     if (!wy::seq_bounds(cu_seqlens, T_total, N, n, t0, t1)) {
         if (tid == 0) raise_flag(flags, KDA_DEVFLAG_CU_SEQLENS);
@@ -136,8 +142,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
     const uint32_t tmem = *slot_tm;
 
     if (warp < 8) {
-        // ---------------- data warps: lane = value column dv, g = half of the accumulator columns
-        const int dv = 32 * (warp & 3) + lane;
+        // ---------------- data warps: lanes 0..15 = value columns (M = 64 accumulator rows),
+        // g = half of the accumulator columns
+        const bool act = lane < 16;
+        const int r = 16 * (warp & 3) + (lane & 15);  // accumulator row = value column within the half
+        const int dv = DVH * half + r;                  // value column
         const int g = warp >> 2;
         const uint32_t tq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {   // S_0^T into state buffer 0 (rows i = 64 g .. 64 g + 63 of S_0)
@@ -147,7 +156,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                 float v[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    v[e] = initial_state ? initial_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] : 0.f;
+                    v[e] = (act && initial_state) ? initial_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] : 0.f;
                 tmem_st32(tq + TM_S + i0, v);
             }
             tmem_st_wait();
@@ -158,22 +167,24 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             if (len == C) {  // whole chunk: rows into the o tile, then one TMA store
                 if (tid == 0) bulk_wait_read();  // the previous tile has left shared memory
                 group_sync(1, DATA_THREADS);
-                if (o_is_f32) {
-                    float* ost = reinterpret_cast<float*>(sm + OFF_OST);
+                if (act) {
+                    if (o_is_f32) {
+                        float* ost = reinterpret_cast<float*>(sm + OFF_OST);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DV + dv] = x[e];
-                } else {
-                    __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OFF_OST);
+                        for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DVH + r] = x[e];
+                    } else {
+                        __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OFF_OST);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DV + dv] = __float2bfloat16_rn(x[e]);
+                        for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DVH + r] = __float2bfloat16_rn(x[e]);
+                    }
                 }
                 fence_async_smem();
                 group_sync(1, DATA_THREADS);
                 if (tid == 0) {
-                    tma_store_3d(&tm_o, sm + OFF_OST, 0, h, static_cast<int>(c0));
+                    tma_store_3d(&tm_o, sm + OFF_OST, DVH * half, h, static_cast<int>(c0));
                     bulk_commit();
                 }
-            } else {  // the sequence's last, partial chunk: its own rows only
+            } else if (act) {  // the sequence's last, partial chunk: its own rows only
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int t = 32 * g + e;
@@ -183,11 +194,16 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
         };
         // this thread's share of chunk c's B^T (rows i = 64 g .. +63) and Uo^T (tokens 32 g .. +31)
         float4 pb[16], pu[8];
+#pragma unroll
+        for (int s = 0; s < 16; ++s) pb[s] = make_float4(0.f, 0.f, 0.f, 0.f);  // lanes 16..31 carry zeros
+#pragma unroll
+        for (int s = 0; s < 8; ++s) pu[s] = make_float4(0.f, 0.f, 0.f, 0.f);
         auto fetch = [&](int c) {
             const float4* rec =
                 reinterpret_cast<const float4*>(ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES);
             const float4* gB = rec + wy::REC_B / 16 + (16 * g) * 128;
             const float4* gU = rec + wy::REC_UO / 16 + (8 * g) * 128;
+            if (!act) return;
 #pragma unroll
             for (int s = 0; s < 16; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
 #pragma unroll
@@ -239,7 +255,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                 float x[32];
                 tmem_ld32(tq + sb + i0, x);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) final_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = x[e];
+                if (act)
+                    for (int e = 0; e < 32; ++e) final_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = x[e];
             }
         }
     } else if (warp == LOADER_WARP) {
@@ -274,8 +291,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t sbase = smem_u32(sm);
-            constexpr uint32_t id_s = idesc_tf32(128, 128, false, false);
-            constexpr uint32_t id_o = idesc_tf32(128, 64, false, false);
+            constexpr uint32_t id_s = idesc_tf32(64, 128, false, false);
+            constexpr uint32_t id_o = idesc_tf32(64, 64, false, false);
             int committed = 0;
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
@@ -323,13 +340,13 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
     CUtensorMap mo;
     const bool f32 = a.dtype_o == KDA_FP32;
     if (!tma_encode_thd(&mo, a.o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2,
-                        DV, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T_total), DV, C,
+                        DV, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T_total), DVH, C,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     cudaError_t err =
         cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    const int64_t blocks = static_cast<int64_t>(a.N) * a.H;
+    const int64_t blocks = static_cast<int64_t>(a.N) * a.H * 2;
     chunk_scan_kernel<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
         mo, static_cast<const unsigned char*>(a.workspace), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
         a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags);
