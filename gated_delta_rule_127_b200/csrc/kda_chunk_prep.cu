@@ -316,29 +316,29 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tma_load_4d(sm + dst, m, 0, static_cast<int>(t.c0), 0, t.h, bar_tma);
     };
 
-    uint32_t loads_issued = 0;  // thread 0: staging loads issued (bar_tma phases)
-    TaskWalker walker;          // thread 0's
+    uint32_t loads_issued = 0;    // thread 0: staging loads issued (bar_tma phases)
+    TaskWalker walker;            // the last thread's: it looks the tasks up
+    constexpr int kWalker = THREADS - 1;
+    if (tid == kWalker) {
+        walker.init(cu_seqlens, T_total, N, H, ws, flags);
+        slots[0] = walker.next();
+        slots[1] = walker.next();
+        slots[2].id = -1;
+    }
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_rest, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_g);
-        walker.init(cu_seqlens, T_total, N, H, ws, flags);
-        const Task t0 = walker.next();
-        Task t1;
-        t1.id = -1;
-        if (t0.id >= 0) {
-            mbar_arrive_expect_tx(bar_tma, kStageBytes);
-            for (int j = 0; j < kLoads; ++j) load_box(t0, j);
-            ++loads_issued;
-            t1 = walker.next();
-        }
-        slots[0] = t0;
-        slots[1] = t1;
-        slots[2].id = -1;
     }
     if (warp == 0) tmem_alloc(slot_tm, TM_COLS);
+    __syncthreads();
+    if (tid == 0 && slots[0].id >= 0) {
+        mbar_arrive_expect_tx(bar_tma, kStageBytes);
+        for (int j = 0; j < kLoads; ++j) load_box(slots[0], j);
+        ++loads_issued;
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -457,7 +457,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mma_tf32_ts(tmem + TM_D1, tmem + TM_A1 + 8 * kk, bkm + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4),
                             id1, kk > 0);
             mma_commit(bar_mma);
-            slots[aft] = walker.next();  // while the tensor cores run: the task after the next
         }
         failed = !mbar_wait(bar_mma, 0, kWaitPolls);  // bar_mma completes twice per task: parities 0, 1
         if (__syncthreads_or(failed)) { failed = true; break; }
@@ -518,25 +517,23 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                          b8 + (((kk >> 2) * 32768 + (kk & 3) * 32) >> 4), id8, kk > 0);
             mma_commit(bar_mma);
         }
+        if (tid == kWalker) slots[aft] = walker.next();  // while MMA 2 runs: the task after the next
         failed = !mbar_wait(bar_mma, 1, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        // [W | U] (M=64 layout: row s = 16 q4 + lane in lanes 0..15), columns 64 qr .. -> MN-major over B8
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
+        {   // [W | U] (M=64 layout: row s = 16 q4 + lane % 16), columns 64 qr + 32 (lane / 16) .. +31
+            // -> MN-major over B8
             float x[32];
-            tmem_ld32(tq + TM_D8 + 64 * qr + 32 * jj, x);
-            if (lane < 16) {
-                const int s = 16 * q4 + lane;
+            tmem_ld32_x2<32>(tq + TM_D8 + 64 * qr, x);
+            const int s = 16 * q4 + (lane & 15);
 #pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) {
-                    const int n0 = 64 * qr + 32 * jj + 8 * e8;
-                    float4* d = reinterpret_cast<float4*>(sm + OFF_B8 + sw32b_off(s, n0, 64));
-                    d[0] = make_float4(to_tf32(x[8 * e8]), to_tf32(x[8 * e8 + 1]), to_tf32(x[8 * e8 + 2]),
-                                       to_tf32(x[8 * e8 + 3]));
-                    d[1] = make_float4(to_tf32(x[8 * e8 + 4]), to_tf32(x[8 * e8 + 5]), to_tf32(x[8 * e8 + 6]),
-                                       to_tf32(x[8 * e8 + 7]));
-                }
+            for (int e8 = 0; e8 < 4; ++e8) {
+                const int n0 = 64 * qr + 32 * (lane >> 4) + 8 * e8;
+                float4* d = reinterpret_cast<float4*>(sm + OFF_B8 + sw32b_off(s, n0, 64));
+                d[0] = make_float4(to_tf32(x[8 * e8]), to_tf32(x[8 * e8 + 1]), to_tf32(x[8 * e8 + 2]),
+                                   to_tf32(x[8 * e8 + 3]));
+                d[1] = make_float4(to_tf32(x[8 * e8 + 4]), to_tf32(x[8 * e8 + 5]), to_tf32(x[8 * e8 + 6]),
+                                   to_tf32(x[8 * e8 + 7]));
             }
         }
         fence_async_smem();
@@ -574,29 +571,43 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         failed = !mbar_wait(bar_rest, it & 1, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        {   // Qh = Q e^G - P W (row t = 16 q4 + lane, channels 32 qr ..) -> staging, K-major rows t
-            const int t = 16 * q4 + lane;
-            const bool live = t < len;
+        {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record, first,
+            // so that the stores drain while the rest of the record is formed
             float x[32];
-            tmem_ld32(tq + TM_PW + 32 * qr, x);
-            if (lane < 16) {
-                unsigned char* row = sm + STG_Q + qr * 8192 + t * 128;  // K-block qr, row t
+            tmem_ld32(tq + TM_BT + 32 * qr, x);
+            float4* gb = reinterpret_cast<float4*>(rec + wy::REC_B);
 #pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) {
-                    const int cc = 32 * qr + 8 * e8;
-                    float qv[8];
-                    unpack8(*reinterpret_cast<const uint4*>(sm + OFF_SQ + bf16_sw_off(t, cc)), qv);
-                    const float4 e0 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc, 64));
-                    const float4 e1 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc + 4, 64));
-                    const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-                    float qh[8];
+            for (int s4 = 0; s4 < 8; ++s4)
+                gb[(8 * qr + s4) * 128 + c] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
+            float y[16];
+            tmem_ld16(tq + TM_UT + 16 * qr, y);
+            float4* gu = reinterpret_cast<float4*>(rec + wy::REC_UO);
 #pragma unroll
-                    for (int w = 0; w < 8; ++w)
-                        qh[w] = to_tf32((live ? qv[w] * ev[w] * x_egm[cc + w] : 0.f) - x[8 * e8 + w]);
-                    *reinterpret_cast<float4*>(row + (((2 * e8) ^ (t & 7)) << 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
-                    *reinterpret_cast<float4*>(row + (((2 * e8 + 1) ^ (t & 7)) << 4)) =
-                        make_float4(qh[4], qh[5], qh[6], qh[7]);
-                }
+            for (int s4 = 0; s4 < 4; ++s4)
+                gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4], y[4 * s4 + 1], y[4 * s4 + 2], y[4 * s4 + 3]);
+        }
+        {   // Qh = Q e^G - P W (row t = 16 q4 + lane % 16, channels 32 qr + 16 (lane / 16) ..) -> staging,
+            // K-major rows t
+            const int t = 16 * q4 + (lane & 15), hc = lane >> 4;
+            const bool live = t < len;
+            float x[16];
+            tmem_ld16_x2<16>(tq + TM_PW + 32 * qr, x);
+            unsigned char* row = sm + STG_Q + qr * 8192 + t * 128;  // K-block qr, row t
+#pragma unroll
+            for (int e8 = 0; e8 < 2; ++e8) {
+                const int cc = 32 * qr + 16 * hc + 8 * e8;
+                float qv[8];
+                unpack8(*reinterpret_cast<const uint4*>(sm + OFF_SQ + bf16_sw_off(t, cc)), qv);
+                const float4 e0 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc, 64));
+                const float4 e1 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc + 4, 64));
+                const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                float qh[8];
+#pragma unroll
+                for (int w = 0; w < 8; ++w)
+                    qh[w] = to_tf32((live ? qv[w] * ev[w] * x_egm[cc + w] : 0.f) - x[8 * e8 + w]);
+                const int ch = 4 * hc + 2 * e8;  // 16-byte chunk of the row within the K-block
+                *reinterpret_cast<float4*>(row + ((ch ^ (t & 7)) << 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
+                *reinterpret_cast<float4*>(row + (((ch + 1) ^ (t & 7)) << 4)) = make_float4(qh[4], qh[5], qh[6], qh[7]);
             }
         }
         const Task tn = slots[nxt];
@@ -619,20 +630,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int u = 0; u < 4; ++u) m[u] = to_tf32((c == 32 * qr + 4 * e4 + u ? gam : 0.f) - x[4 * e4 + u]);
                 *reinterpret_cast<float4*>(row + ((e4 ^ (c & 7)) << 4)) = make_float4(m[0], m[1], m[2], m[3]);
             }
-        }
-        {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record
-            float x[32];
-            tmem_ld32(tq + TM_BT + 32 * qr, x);
-            float4* gb = reinterpret_cast<float4*>(rec + wy::REC_B);
-#pragma unroll
-            for (int s4 = 0; s4 < 8; ++s4)
-                gb[(8 * qr + s4) * 128 + c] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
-            float y[16];
-            tmem_ld16(tq + TM_UT + 16 * qr, y);
-            float4* gu = reinterpret_cast<float4*>(rec + wy::REC_UO);
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4)
-                gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4], y[4 * s4 + 1], y[4 * s4 + 2], y[4 * s4 + 3]);
         }
         fence_async_smem();
         tc_fence_before_sync();
