@@ -63,7 +63,7 @@ constexpr uint32_t OFF_MISC = 212992;  // beta[2][64] (this task, the next), qua
                                        //   g_m, g_C, e^{g_m}, e^{g_C} [128]
 constexpr uint32_t OFF_X = 217600;     // 32 x 32 fp32 scratch for the inverse
 constexpr uint32_t OFF_TASK = 221696;  // three Task slots (this task, the next, the one after)
-constexpr uint32_t OFF_BARS = 221792;  // mbarriers: TMA, MMAs 1-2, MMAs 3-6; then the TMEM base address
+constexpr uint32_t OFF_BARS = 221792;  // mbarriers: TMA, MMAs 1-2, MMAs 3-4, MMAs 5-6; then the TMEM base address
 constexpr uint32_t SMEM_USED = 221832;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 // after MMA 1 (k, v staging and K- are dead):
@@ -301,7 +301,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     Task* slots = reinterpret_cast<Task*>(sm + OFF_TASK);  // ring of 3: this task, the next, the one after
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     uint64_t* bar_mma = bar_tma + 1;   // MMAs 1 and 2
-    uint64_t* bar_rest = bar_tma + 2;  // MMAs 3-6
+    uint64_t* bar_rest = bar_tma + 2;  // MMAs 3-4
+    uint64_t* bar_bu = bar_tma + 3;    // MMAs 5-6
     uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 32);
 
     constexpr uint32_t kGateBytes = C * DK * sizeof(TG);
@@ -329,6 +330,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_rest, 1);
+        mbar_init(bar_bu, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_g);
     }
@@ -553,26 +555,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             constexpr uint32_t id_kw = idesc_tf32(128, 128, false, true);
             constexpr uint32_t id_bt = idesc_tf32(128, 128, true, false);
             constexpr uint32_t id_ut = idesc_tf32(128, 64, true, false);
-#pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)
-                mma_tf32(tmem + TM_PW, dp + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), bw + static_cast<uint64_t>(kk) * 64,
-                         id_pw, kk > 0);
+            // B^T and Uo^T first: their read-out and stores to the record overlap MMAs 3 and 4
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk) {
-                const uint64_t kt = dkt + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-                const uint64_t pp = dp + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
                 const uint64_t mn = static_cast<uint64_t>(kk) * 64;
-                mma_tf32(tmem + TM_KW, kt, bw + mn, id_kw, kk > 0);
-                mma_tf32(tmem + TM_BT, au + mn, kt, id_bt, kk > 0);
-                mma_tf32(tmem + TM_UT, au + mn, pp, id_ut, kk > 0);
+                mma_tf32(tmem + TM_BT, au + mn, dkt + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), id_bt, kk > 0);
+                mma_tf32(tmem + TM_UT, au + mn, dp + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_ut, kk > 0);
+            }
+            mma_commit(bar_bu);
+#pragma unroll
+            for (int kk = 0; kk < C / 8; ++kk) {
+                const uint64_t mn = static_cast<uint64_t>(kk) * 64;
+                mma_tf32(tmem + TM_PW, dp + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), bw + mn, id_pw, kk > 0);
+                mma_tf32(tmem + TM_KW, dkt + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), bw + mn, id_kw, kk > 0);
             }
             mma_commit(bar_rest);
         }
-        failed = !mbar_wait(bar_rest, it & 1, kWaitPolls);
+        failed = !mbar_wait(bar_bu, it & 1, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record, first,
-            // so that the stores drain while the rest of the record is formed
+        {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record
             float x[32];
             tmem_ld32(tq + TM_BT + 32 * qr, x);
             float4* gb = reinterpret_cast<float4*>(rec + wy::REC_B);
@@ -586,6 +588,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int s4 = 0; s4 < 4; ++s4)
                 gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4], y[4 * s4 + 1], y[4 * s4 + 2], y[4 * s4 + 3]);
         }
+        failed = !mbar_wait(bar_rest, it & 1, kWaitPolls);
+        if (__syncthreads_or(failed)) { failed = true; break; }
+        tc_fence_after_sync();
         {   // Qh = Q e^G - P W (row t = 16 q4 + lane % 16, channels 32 qr + 16 (lane / 16) ..) -> staging,
             // K-major rows t
             const int t = 16 * q4 + (lane & 15), hc = lane >> 4;

@@ -18,10 +18,11 @@
 // fp32; it is stored in fp32 at the end.
 //
 // Roles (320 threads): warps 0-7 fill the accumulators and write o (through a shared-memory tile and
-// one TMA store per full chunk) and the final state -- lanes 0..15 of warp w serve the value columns
-// 16 (w % 4) .. +15 of the CTA's half (the M = 64 accumulator rows, tensor-memory lanes 32 (w % 4) ..
-// +15) and half w / 4 of the accumulator columns, and hold the next chunk's share of B and Uo in
-// registers while the current chunk's MMAs run; warp 8 lane 0 brings each chunk's Mt and Qh operand tiles into a two-stage
+// one TMA store per full chunk) and the final state -- warp w serves the value columns 16 (w % 4) ..
+// +15 of the CTA's half (the M = 64 accumulator rows, tensor-memory lanes 32 (w % 4) .. +15; its lanes
+// 16..31 reach the same rows through the 16x32bx2 access shape at a column offset) and half w / 4 of
+// the accumulator columns, and holds the next chunk's share of B and Uo in registers while the
+// current chunk's MMAs run; warp 8 lane 0 brings each chunk's Mt and Qh operand tiles into a two-stage
 // shared-memory ring with bulk copies (and asks L2 for the B and Uo of the chunk after); warp 9
 // lane 0 issues the MMAs.
 // Tensor memory: three state buffers (S_n read while S_{n+1} accumulates and S_{n+2}'s B is written)
@@ -142,41 +143,37 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
     const uint32_t tmem = *slot_tm;
 
     if (warp < 8) {
-        // ---------------- data warps: lanes 0..15 = value columns (M = 64 accumulator rows),
-        // g = half of the accumulator columns
-        const bool act = lane < 16;
+        // ---------------- data warps: warp w serves the accumulator rows (value columns) 16 (w % 4) ..
+        // +15, lanes 0..15 and 16..31 two column ranges of half g = w / 4 of the accumulator columns
+        const int hl = lane >> 4;                       // second copy of the warp's 16 rows
         const int r = 16 * (warp & 3) + (lane & 15);  // accumulator row = value column within the half
         const int dv = DVH * half + r;                  // value column
         const int g = warp >> 2;
         const uint32_t tq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        {   // S_0^T into state buffer 0 (rows i = 64 g .. 64 g + 63 of S_0)
+        {   // S_0^T into state buffer 0: this lane's rows i = 64 g + 32 hl .. +31 of S_0
+            const int i0 = 64 * g + 32 * hl;
+            float v[32];
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int i0 = 64 * g + 32 * jj;
-                float v[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    v[e] = (act && initial_state) ? initial_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] : 0.f;
-                tmem_st32(tq + TM_S + i0, v);
-            }
+            for (int e = 0; e < 32; ++e)
+                v[e] = initial_state ? initial_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] : 0.f;
+            tmem_st32_x2<32>(tq + TM_S + 64 * g, v);
             tmem_st_wait();
         }
-        auto emit_o = [&](int c, const float (&x)[32]) {  // tokens 32 g .. 32 g + 31 of O_c -> o
+        auto emit_o = [&](int c, const float (&x)[16]) {  // tokens 32 g + 16 hl .. +15 of O_c -> o
             const int64_t c0 = t0 + static_cast<int64_t>(c) * C;
             const int len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
+            const int tb = 32 * g + 16 * hl;
             if (len == C) {  // whole chunk: rows into the o tile, then one TMA store
                 if (tid == 0) bulk_wait_read();  // the previous tile has left shared memory
                 group_sync(1, DATA_THREADS);
-                if (act) {
-                    if (o_is_f32) {
-                        float* ost = reinterpret_cast<float*>(sm + OFF_OST);
+                if (o_is_f32) {
+                    float* ost = reinterpret_cast<float*>(sm + OFF_OST);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DVH + r] = x[e];
-                    } else {
-                        __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OFF_OST);
+                    for (int e = 0; e < 16; ++e) ost[(tb + e) * DVH + r] = x[e];
+                } else {
+                    __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OFF_OST);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ost[(32 * g + e) * DVH + r] = __float2bfloat16_rn(x[e]);
-                    }
+                    for (int e = 0; e < 16; ++e) ost[(tb + e) * DVH + r] = __float2bfloat16_rn(x[e]);
                 }
                 fence_async_smem();
                 group_sync(1, DATA_THREADS);
@@ -184,55 +181,50 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                     tma_store_3d(&tm_o, sm + OFF_OST, DVH * half, h, static_cast<int>(c0));
                     bulk_commit();
                 }
-            } else if (act) {  // the sequence's last, partial chunk: its own rows only
+            } else {  // the sequence's last, partial chunk: its own rows only
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = 32 * g + e;
-                    if (t < len) store_o(o_ptr, ((c0 + t) * H + h) * DV + dv, x[e], o_is_f32 != 0);
-                }
+                for (int e = 0; e < 16; ++e)
+                    if (tb + e < len) store_o(o_ptr, ((c0 + tb + e) * H + h) * DV + dv, x[e], o_is_f32 != 0);
             }
         };
-        // this thread's share of chunk c's B^T (rows i = 64 g .. +63) and Uo^T (tokens 32 g .. +31)
-        float4 pb[16], pu[8];
-#pragma unroll
-        for (int s = 0; s < 16; ++s) pb[s] = make_float4(0.f, 0.f, 0.f, 0.f);  // lanes 16..31 carry zeros
-#pragma unroll
-        for (int s = 0; s < 8; ++s) pu[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+        // this lane's share of chunk c's B^T (rows i = 64 g + 32 hl .. +31) and Uo^T (tokens 32 g + 16 hl
+        // .. +15), loaded one chunk ahead
+        float4 pb[8], pu[4];
         auto fetch = [&](int c) {
             const float4* rec =
                 reinterpret_cast<const float4*>(ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES);
-            const float4* gB = rec + wy::REC_B / 16 + (16 * g) * 128;
-            const float4* gU = rec + wy::REC_UO / 16 + (8 * g) * 128;
-            if (!act) return;
+            const float4* gB = rec + wy::REC_B / 16 + (16 * g + 8 * hl) * 128;
+            const float4* gU = rec + wy::REC_UO / 16 + (8 * g + 4 * hl) * 128;
 #pragma unroll
-            for (int s = 0; s < 16; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
+            for (int s = 0; s < 8; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) pu[s] = __ldcs(gU + s * 128 + dv);
-        };
-        auto put32 = [&](uint32_t taddr, const float4* p) {
-            float v[32];
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                v[4 * s] = p[s].x; v[4 * s + 1] = p[s].y; v[4 * s + 2] = p[s].z; v[4 * s + 3] = p[s].w;
-            }
-            tmem_st32(taddr, v);
+            for (int s = 0; s < 4; ++s) pu[s] = __ldcs(gU + s * 128 + dv);
         };
         bool ok = true;
         if (nc > 0) fetch(0);
         for (int c = 0; c < nc && ok; ++c) {
             // O_{c-2} out of output buffer c & 1 first, so chunk c's accumulators can be signalled before
             // O_{c-2} is written to memory
-            float ox[32];
+            float ox[16];
             if (c >= 2) {
                 ok = wait_or_abort(odone + (c & 1), ((c - 2) >> 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after_sync();
-                tmem_ld32(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
+                tmem_ld16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
             }
-            const uint32_t sb = TM_S + 128 * ((c + 1) % 3) + 64 * g;
-            put32(tq + sb, pb);
-            put32(tq + sb + 32, pb + 8);
-            put32(tq + TM_O + 64 * (c & 1) + 32 * g, pu);
+            {
+                float vb[32], vu[16];
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    vb[4 * s] = pb[s].x; vb[4 * s + 1] = pb[s].y; vb[4 * s + 2] = pb[s].z; vb[4 * s + 3] = pb[s].w;
+                }
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    vu[4 * s] = pu[s].x; vu[4 * s + 1] = pu[s].y; vu[4 * s + 2] = pu[s].z; vu[4 * s + 3] = pu[s].w;
+                }
+                tmem_st32_x2<32>(tq + TM_S + 128 * ((c + 1) % 3) + 64 * g, vb);
+                tmem_st16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, vu);
+            }
             tmem_st_wait();
             tc_fence_before_sync();
             mbar_arrive(sinit + (c & 1));
@@ -243,21 +235,16 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             ok = wait_or_abort(odone + (c & 1), (c >> 1) & 1, abort);
             if (!ok) break;
             tc_fence_after_sync();
-            float ox[32];
-            tmem_ld32(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
+            float ox[16];
+            tmem_ld16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
             emit_o(c, ox);
         }
         if (ok && final_state) {  // after the last output MMA, the last state MMA is complete too
-            const uint32_t sb = TM_S + 128 * (nc % 3);
+            const int i0 = 64 * g + 32 * hl;
+            float x[32];
+            tmem_ld32_x2<32>(tq + TM_S + 128 * (nc % 3) + 64 * g, x);
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int i0 = 64 * g + 32 * jj;
-                float x[32];
-                tmem_ld32(tq + sb + i0, x);
-#pragma unroll
-                if (act)
-                    for (int e = 0; e < 32; ++e) final_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = x[e];
-            }
+            for (int e = 0; e < 32; ++e) final_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = x[e];
         }
     } else if (warp == LOADER_WARP) {
         // ---------------- loader: chunk c's Mt and Qh tiles into stage c & 1
