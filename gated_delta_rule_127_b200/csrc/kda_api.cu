@@ -42,22 +42,12 @@ size_t dtype_size(kda_dtype d) { return d == KDA_FP32 ? 4 : 2; }
 bool supported_dim(int d) { return d == 64 || d == 128; }
 
 }  // namespace
-}  // namespace kda
 
-extern "C" {
-
-size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int dk, int dv, int chunk_size) {
-    (void)chunk_size;
-    if (T_total < 0 || N <= 0 || H <= 0) return 0;
-    return kda::chunk_wy_workspace_size(T_total, N, H, dk, dv);
-}
-
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
-                         const void* beta, const float* initial_state, const int32_t* cu_seqlens,
-                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
-                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
-                         float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
-    using namespace kda;
+// kda_chunk_fwd and kda_gdn_chunk_fwd: scalar_gate selects a [T_total, H] log_alpha.
+kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                     const float* initial_state, const int32_t* cu_seqlens, int64_t T_total, int N, int H, int dk,
+                     int dv, int chunk_size, kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                     float* final_state, void* workspace, size_t workspace_bytes, void* stream, bool scalar_gate) {
     if (T_total < 0 || N <= 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk_size <= 0)
         return KDA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
@@ -67,14 +57,15 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     if ((int64_t)N * H * (dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     if (T_total > 0) {
         if (!q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
-        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KDA_ERR_INVALID_ARG;
+        if (scalar_gate ? !aligned_to(log_alpha, dtype_size(dtype_gate)) : !aligned16(log_alpha))
             return KDA_ERR_INVALID_ARG;
         if (!aligned_to(beta, dtype_size(dtype_gate))) return KDA_ERR_INVALID_ARG;
     }
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_INVALID_ARG;
     if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
-    const size_t need = kda_chunk_fwd_workspace_size(T_total, N, H, dk, dv, chunk_size);
+    const size_t need = (T_total < 0 || N <= 0 || H <= 0) ? 0 : chunk_wy_workspace_size(T_total, N, H, dk, dv);
     const bool have_ws = workspace != nullptr && workspace_bytes > 0;
     if (have_ws && (workspace_bytes < need || !aligned16(workspace))) return KDA_ERR_INVALID_ARG;
 
@@ -85,6 +76,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     a.dtype_qkv = dtype_qkv; a.dtype_gate = dtype_gate; a.dtype_o = dtype_o;
     a.o = o; a.final_state = final_state; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     a.stream = static_cast<cudaStream_t>(stream);
+    a.scalar_gate = scalar_gate;
     if (device_flags_ptr(&a.flags) != cudaSuccess) return KDA_ERR_CUDA;
 
     cudaError_t err;
@@ -99,11 +91,10 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
-                           const void* beta, float* state, int B, int H, int dk, int dv,
-                           kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
-                           void* stream) {
-    using namespace kda;
+// kda_decode_step and kda_gdn_decode_step: scalar_gate selects a [B, H] log_alpha.
+kda_status decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                       float* state, int B, int H, int dk, int dv, kda_dtype dtype_qkv, kda_dtype dtype_gate,
+                       kda_dtype dtype_o, void* o, void* stream, bool scalar_gate) {
     if (B < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
         return KDA_ERR_INVALID_ARG;
@@ -122,7 +113,52 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const vo
     a.dtype_qkv = dtype_qkv; a.dtype_gate = dtype_gate; a.dtype_o = dtype_o; a.o = o;
     a.stream = static_cast<cudaStream_t>(stream);
     a.flags = nullptr;
+    a.scalar_gate = scalar_gate;
     return launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace kda
+
+extern "C" {
+
+size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int dk, int dv, int chunk_size) {
+    (void)chunk_size;
+    if (T_total < 0 || N <= 0 || H <= 0) return 0;
+    return kda::chunk_wy_workspace_size(T_total, N, H, dk, dv);
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
+                         const void* beta, const float* initial_state, const int32_t* cu_seqlens,
+                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                         float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+    return kda::chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, T_total, N, H, dk, dv, chunk_size,
+                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, false);
+}
+
+kda_status kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
+                             const void* beta, const float* initial_state, const int32_t* cu_seqlens,
+                             int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                             kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                             float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+    return kda::chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, T_total, N, H, dk, dv, chunk_size,
+                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, true);
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
+                           const void* beta, float* state, int B, int H, int dk, int dv,
+                           kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                           void* stream) {
+    return kda::decode_step(q, k, v, log_alpha, beta, state, B, H, dk, dv, dtype_qkv, dtype_gate, dtype_o, o,
+                            stream, false);
+}
+
+kda_status kda_gdn_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
+                               const void* beta, float* state, int B, int H, int dk, int dv,
+                               kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                               void* stream) {
+    return kda::decode_step(q, k, v, log_alpha, beta, state, B, H, dk, dv, dtype_qkv, dtype_gate, dtype_o, o,
+                            stream, true);
 }
 
 kda_status kda_get_device_status(void* stream, uint32_t* flags) {

@@ -64,7 +64,8 @@ constexpr uint32_t OFF_MISC = 212992;  // beta[2][64] (this task, the next), qua
 constexpr uint32_t OFF_X = 217600;     // 32 x 32 fp32 scratch for the inverse
 constexpr uint32_t OFF_TASK = 221696;  // three Task slots (this task, the next, the one after)
 constexpr uint32_t OFF_BARS = 221792;  // mbarriers: TMA, MMAs 1-2, MMAs 3-4, MMAs 5-6; then the TMEM base address
-constexpr uint32_t SMEM_USED = 221832;
+constexpr uint32_t OFF_SAL = 221840;   // scalar log-decay [2][64] (Gated DeltaNet gates), by task parity
+constexpr uint32_t SMEM_USED = OFF_SAL + 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 // after MMA 1 (k, v staging and K- are dead):
 constexpr uint32_t OFF_A = 49152;      // A fp32 [64][TP]
@@ -277,12 +278,15 @@ __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, f
     __syncthreads();
 }
 
-template <typename TG>
+// SG: Gated DeltaNet gates -- log_alpha is [T_total, H], one decay rate per token and head, read
+// with beta and broadcast over the key channels (tm_g is then unused).
+template <typename TG, bool SG>
 __global__ void __launch_bounds__(THREADS, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                  const TG* __restrict__ beta, const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N,
-                  int H, unsigned char* __restrict__ ws, unsigned int* flags) {
+                  const TG* __restrict__ beta, const TG* __restrict__ log_alpha_sg,
+                  const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H,
+                  unsigned char* __restrict__ ws, unsigned int* flags) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;   // tensor-memory lane quadrant
     const int qr = warp >> 2;  // row quarter (elementwise pass) / column quarter (read-outs)
@@ -297,6 +301,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float* x_gc = x_gm + 128;
     float* x_egm = x_gc + 128;
     float* x_gam = x_egm + 128;
+    float* s_alpha2 = reinterpret_cast<float*>(sm + OFF_SAL);  // [2][64] (SG only)
     float* xs = reinterpret_cast<float*>(sm + OFF_X);
     Task* slots = reinterpret_cast<Task*>(sm + OFF_TASK);  // ring of 3: this task, the next, the one after
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
@@ -305,12 +310,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t* bar_bu = bar_tma + 3;    // MMAs 5-6
     uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 32);
 
-    constexpr uint32_t kGateBytes = C * DK * sizeof(TG);
+    constexpr uint32_t kGateBytes = SG ? 0 : C * DK * sizeof(TG);
     constexpr uint32_t kStageBytes = 3 * C * DK * 2 + kGateBytes;
     // Tile j (k, q, v, log_alpha) of a task into the staging buffers: one box covering all of the
     // tile's 128-byte column blocks (completion on bar_tma, whose expected byte count kStageBytes is
     // set once per task).  The four are issued by different warps.
-    constexpr int kLoads = 4;
+    constexpr int kLoads = SG ? 3 : 4;
     auto load_box = [&](const Task& t, int j) {
         const CUtensorMap* m = j == 0 ? &tm_k : j == 1 ? &tm_q : j == 2 ? &tm_v : &tm_g;
         const uint32_t dst = j == 0 ? OFF_SK : j == 1 ? OFF_SQ : j == 2 ? OFF_SV : OFF_G + (sizeof(TG) == 4 ? 0u : 16384u);
@@ -332,7 +337,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(bar_rest, 1);
         mbar_init(bar_bu, 1);
         fence_mbar_init();
-        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_g);
+        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
+        if (!SG) tma_prefetch_desc(&tm_g);
     }
     if (warp == 0) tmem_alloc(slot_tm, TM_COLS);
     __syncthreads();
@@ -348,11 +354,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tq = tmem + (static_cast<uint32_t>(q4 * 32) << 16);  // this warp's lane quadrant
     const int c = 32 * q4 + lane;  // key channel (elementwise pass) and tensor-memory lane
     bool failed = false;
-    // beta of a task into s_beta2[parity] (threads 64..127; later read only after a barrier)
+    // beta of a task into s_beta2[parity] (threads 64..127), and with SG its scalar log-decay into
+    // s_alpha2[parity] (threads 0..63); both are read only after a barrier
     auto load_beta = [&](const Task& t, uint32_t parity) {
         const int r = tid - 64;
         if (r >= 0 && r < C && t.id >= 0)
             s_beta2[64 * parity + r] = r < t.len ? to_f32(beta[(t.c0 + r) * H + t.h]) : 0.f;
+        if (SG && tid < C && t.id >= 0)
+            s_alpha2[64 * parity + tid] = tid < t.len ? to_f32(log_alpha_sg[(t.c0 + tid) * H + t.h]) : 0.f;
     };
     load_beta(slots[0], 0);  // (slots are written by thread 0 before the barrier above)
     __syncthreads();
@@ -375,7 +384,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             float run = 0.f;
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                run += (rb + r) < len ? gate_at<TG>(sm, rb + r, c) : 0.f;
+                run += (rb + r) < len ? (SG ? s_alpha2[64 * (it & 1) + rb + r] : gate_at<TG>(sm, rb + r, c)) : 0.f;
                 g[r] = run;
             }
             x_part[qr * 128 + c] = run;
@@ -669,7 +678,7 @@ int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <typename TG>
+template <typename TG, bool SG>
 cudaError_t launch_prep(const ChunkArgs& a) {
     CUtensorMap mq, mk, mv, mg;
     const uint64_t T = static_cast<uint64_t>(a.T_total), H = static_cast<uint64_t>(a.H);
@@ -681,15 +690,17 @@ cudaError_t launch_prep(const ChunkArgs& a) {
     if (!tma_encode_blocks(&mq, a.q, bf, 2, DK, H, T, 64, C, sw) ||
         !tma_encode_blocks(&mk, a.k, bf, 2, DK, H, T, 64, C, sw) ||
         !tma_encode_blocks(&mv, a.v, bf, 2, DV, H, T, 64, C, sw) ||
-        !tma_encode_blocks(&mg, a.log_alpha, gdt, sizeof(TG), DK, H, T, gblk, C, sw))
+        (!SG && !tma_encode_blocks(&mg, a.log_alpha, gdt, sizeof(TG), DK, H, T, gblk, C, sw)))
         return cudaErrorInvalidValue;
-    auto kern = chunk_prep_kernel<TG>;
+    if (SG) mg = mq;  // not read
+    auto kern = chunk_prep_kernel<TG, SG>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int64_t ntasks = wy::num_slots(a.T_total, a.N) * a.H;
     const int64_t sms = sm_count();
     const unsigned grid = static_cast<unsigned>(ntasks < sms ? ntasks : sms);
-    kern<<<grid, THREADS, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, static_cast<const TG*>(a.beta), a.cu_seqlens,
+    kern<<<grid, THREADS, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, static_cast<const TG*>(a.beta),
+                                                  SG ? static_cast<const TG*>(a.log_alpha) : nullptr, a.cu_seqlens,
                                                   a.T_total, a.N, a.H, static_cast<unsigned char*>(a.workspace),
                                                   a.flags);
     return cudaGetLastError();
@@ -703,7 +714,8 @@ size_t chunk_wy_workspace_size(int64_t T_total, int N, int H, int dk, int dv) {
 }
 
 cudaError_t launch_chunk_prep(const ChunkArgs& a) {
-    return a.dtype_gate == KDA_FP32 ? launch_prep<float>(a) : launch_prep<__nv_bfloat16>(a);
+    if (a.scalar_gate) return a.dtype_gate == KDA_FP32 ? launch_prep<float, true>(a) : launch_prep<__nv_bfloat16, true>(a);
+    return a.dtype_gate == KDA_FP32 ? launch_prep<float, false>(a) : launch_prep<__nv_bfloat16, false>(a);
 }
 
 }  // namespace kda

@@ -100,7 +100,7 @@ chunk_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
                   const TG* __restrict__ log_alpha, const TG* __restrict__ beta,
                   const float* initial_state, const int32_t* __restrict__ cu_seqlens,
                   int64_t T_total, int N, int H, int DV, TO* __restrict__ o, float* final_state,
-                  unsigned int* flags) {
+                  unsigned int* flags, int scalar_gate) {
     using Sm = SimtSmem<DK>;
     constexpr int KP = Sm::KP;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -147,7 +147,8 @@ chunk_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
             float kv = 0.f, qv = 0.f, av = 0.f;
             if (r < len) {
                 const int64_t off = (c0 + r) * qk_row + (int64_t)h * DK + c;
-                kv = to_f32(k[off]); qv = to_f32(q[off]); av = to_f32(log_alpha[off]);
+                kv = to_f32(k[off]); qv = to_f32(q[off]);
+                av = to_f32(log_alpha[scalar_gate ? (c0 + r) * H + h : off]);  // GDN: one rate per (t, h)
             }
             s.kx[r * KP + c] = kv; s.qx[r * KP + c] = qv; s.gx[r * KP + c] = av;
         }
@@ -299,7 +300,8 @@ cudaError_t launch_typed(const ChunkArgs& a) {
     kern<<<(unsigned)blocks, THREADS, smem, a.stream>>>(
         static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.v),
         static_cast<const TG*>(a.log_alpha), static_cast<const TG*>(a.beta), a.initial_state,
-        a.cu_seqlens, a.T_total, a.N, a.H, a.dv, static_cast<TO*>(a.o), a.final_state, a.flags);
+        a.cu_seqlens, a.T_total, a.N, a.H, a.dv, static_cast<TO*>(a.o), a.final_state, a.flags,
+        a.scalar_gate ? 1 : 0);
     return cudaGetLastError();
 }
 

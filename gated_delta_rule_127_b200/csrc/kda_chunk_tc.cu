@@ -202,11 +202,14 @@ __device__ __forceinline__ void store_row8<__nv_bfloat16>(__nv_bfloat16* dst, co
     *reinterpret_cast<uint4*>(dst) = u;
 }
 
-template <typename TG>
+// SG: Gated DeltaNet gates -- log_alpha is [T_total, H], one decay rate per token and head, read
+// with beta and broadcast over the key channels (tm_la is then unused).
+template <typename TG, bool SG>
 __global__ void __launch_bounds__(THREADS, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
-                const TG* __restrict__ beta, const float* initial_state, const int32_t* __restrict__ cu_seqlens,
+                const TG* __restrict__ beta, const TG* __restrict__ log_alpha_sg,
+                const float* initial_state, const int32_t* __restrict__ cu_seqlens,
                 int64_t T_total, int N, int H, void* __restrict__ o_ptr, int o_is_f32, float* final_state,
                 unsigned int* flags) {
     extern __shared__ unsigned char smem_raw[];
@@ -246,19 +249,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         t0 = static_cast<int64_t>(n) * L;
         t1 = t0 + L;
     }
-    constexpr uint32_t kStageBytes = 2 * C * DK * 2 + C * DK * sizeof(TG) + C * DVS * 2;
+    constexpr uint32_t kStageBytes = 2 * C * DK * 2 + (SG ? 0 : C * DK * sizeof(TG)) + C * DVS * 2;
 
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar2, 1);
         mbar_init(tbar, 1);
         fence_mbar_init();
-        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_la); tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
+        if (!SG) tma_prefetch_desc(&tm_la);
         if (t0 < t1) {
             mbar_arrive_expect_tx(tbar, kStageBytes);
             tma_load_3d(sm + OFF_SK, &tm_k, 0, h, static_cast<int>(t0), tbar);
             tma_load_3d(sm + OFF_SQ, &tm_q, 0, h, static_cast<int>(t0), tbar);
-            tma_load_3d(sm + OFF_SLA, &tm_la, 0, h, static_cast<int>(t0), tbar);
+            if (!SG) tma_load_3d(sm + OFF_SLA, &tm_la, 0, h, static_cast<int>(t0), tbar);
             tma_load_3d(sm + OFF_SV, &tm_v, col0, h, static_cast<int>(t0), tbar);
         }
     }
@@ -287,8 +291,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 8; ++j) S[j] = 0.f;
     }
-    float beta_next = 0.f;
+    float beta_next = 0.f, alpha_next = 0.f;  // alpha_next: SG only
     if (tid < C && t0 + tid < t1) beta_next = to_f32(beta[(t0 + tid) * H + h]);
+    if (SG && tid < C && t0 + tid < t1) alpha_next = to_f32(log_alpha_sg[(t0 + tid) * H + h]);
 
     // Matrix descriptors at K-step 0; K-step kk adds its byte offset >> 4 to the start-address field.
     const uint64_t d_kq = sw128b32_desc(sbase + OFF_KQ, 128 * 128, 512);      // [K+|Q+]^T, MN-major
@@ -303,6 +308,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int64_t c0 = t0; c0 < t1; c0 += C) {
         const int len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
         if (tid < C) s_beta[tid] = beta_next;
+        if (SG && tid < C) tile(sm, OFF_SLA)[tid] = alpha_next;  // the gate staging area holds them
         timed_out = !mbar_wait(tbar, tphase, kWaitPolls);
         if (__syncthreads_or(timed_out)) break;
         tphase ^= 1;
@@ -318,7 +324,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             float run = 0.f;
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                run += (rb + r) < len ? to_f32(sla[(rb + r) * DK + c]) : 0.f;
+                run += (rb + r) < len ? (SG ? tile(sm, OFF_SLA)[rb + r] : to_f32(sla[(rb + r) * DK + c])) : 0.f;
                 g[r] = run;
             }
             x_part[qr * 128 + c] = run;
@@ -386,11 +392,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_arrive_expect_tx(tbar, kStageBytes);
             tma_load_3d(sm + OFF_SK, &tm_k, 0, h, static_cast<int>(c1), tbar);
             tma_load_3d(sm + OFF_SQ, &tm_q, 0, h, static_cast<int>(c1), tbar);
-            tma_load_3d(sm + OFF_SLA, &tm_la, 0, h, static_cast<int>(c1), tbar);
+            if (!SG) tma_load_3d(sm + OFF_SLA, &tm_la, 0, h, static_cast<int>(c1), tbar);
             tma_load_3d(sm + OFF_SV, &tm_v, col0, h, static_cast<int>(c1), tbar);
         }
         tma_pending = c1 < t1;
         if (tid < C) beta_next = (c1 + tid < t1) ? to_f32(beta[(c1 + tid) * H + h]) : 0.f;
+        if (SG && tid < C) alpha_next = (c1 + tid < t1) ? to_f32(log_alpha_sg[(c1 + tid) * H + h]) : 0.f;
 
         // ---- MMA batch 1: [A_raw; P] = [K+; Q+] (K-)^T,  Z = K+ S',  O = Q+ S'
         if (tid == 0) {
@@ -541,22 +548,24 @@ bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TG>
+template <typename TG, bool SG>
 cudaError_t launch_typed(const ChunkArgs& a) {
     CUtensorMap mq, mk, mla, mv;
     const uint64_t T = static_cast<uint64_t>(a.T_total), H = static_cast<uint64_t>(a.H);
     const CUtensorMapDataType gdt = sizeof(TG) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!encode_3d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, H, T, DK, C) ||
         !encode_3d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, H, T, DK, C) ||
-        !encode_3d(&mla, a.log_alpha, gdt, sizeof(TG), DK, H, T, DK, C) ||
+        (!SG && !encode_3d(&mla, a.log_alpha, gdt, sizeof(TG), DK, H, T, DK, C)) ||
         !encode_3d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, H, T, DVS, C))
         return cudaErrorInvalidValue;
-    auto kern = chunk_tc_kernel<TG>;
+    if (SG) mla = mq;  // not read
+    auto kern = chunk_tc_kernel<TG, SG>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int64_t blocks = static_cast<int64_t>(a.N) * a.H * (DV / DVS);
     kern<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
-        mq, mk, mla, mv, static_cast<const TG*>(a.beta), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
+        mq, mk, mla, mv, static_cast<const TG*>(a.beta), SG ? static_cast<const TG*>(a.log_alpha) : nullptr,
+        a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
         a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags);
     return cudaGetLastError();
 }
@@ -569,7 +578,8 @@ bool chunk_tc_supported(const ChunkArgs& a) {
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs& a) {
-    return a.dtype_gate == KDA_FP32 ? launch_typed<float>(a) : launch_typed<__nv_bfloat16>(a);
+    if (a.scalar_gate) return a.dtype_gate == KDA_FP32 ? launch_typed<float, true>(a) : launch_typed<__nv_bfloat16, true>(a);
+    return a.dtype_gate == KDA_FP32 ? launch_typed<float, false>(a) : launch_typed<__nv_bfloat16, false>(a);
 }
 
 

@@ -29,7 +29,7 @@ template <int DK, int DV, typename TIn, typename TG, typename TO>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, 2)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                    const TG* __restrict__ log_alpha, const TG* __restrict__ beta,
-                   float* __restrict__ state, TO* __restrict__ o) {
+                   float* __restrict__ state, TO* __restrict__ o, int scalar_gate) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int TPR = Sh::TPR, RG = Sh::RG, RPT = Sh::RPT;
 
@@ -53,7 +53,7 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     for (int c = tid; c < DK; c += Sh::THREADS) {
         s_k[c] = to_f32(k[u * DK + c]);
         s_q[c] = to_f32(q[u * DK + c]);
-        s_alpha[c] = expf(to_f32(log_alpha[u * DK + c]));
+        s_alpha[c] = expf(to_f32(log_alpha[scalar_gate ? u : u * DK + c]));  // GDN: one rate per (b, h)
     }
     for (int j = tid; j < DV; j += Sh::THREADS) s_v[j] = to_f32(v[u * DV + j]);
     const float b = to_f32(beta[u]);
@@ -106,7 +106,7 @@ cudaError_t launch_typed(const DecodeArgs& a) {
     decode_step_kernel<DK, DV, TIn, TG, TO><<<a.B * a.H, Sh::THREADS, 0, a.stream>>>(
         static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.v),
         static_cast<const TG*>(a.log_alpha), static_cast<const TG*>(a.beta), a.state,
-        static_cast<TO*>(a.o));
+        static_cast<TO*>(a.o), a.scalar_gate ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -25,6 +25,7 @@ struct ChunkArgs {
     size_t workspace_bytes;
     unsigned int* flags;  // device address of the sticky flag word
     cudaStream_t stream;
+    bool scalar_gate;     // log_alpha is [T_total, H] (Gated DeltaNet), broadcast over dk
 };
 
 struct DecodeArgs {
@@ -39,6 +40,7 @@ struct DecodeArgs {
     void* o;
     unsigned int* flags;
     cudaStream_t stream;
+    bool scalar_gate;  // log_alpha is [B, H] (Gated DeltaNet), broadcast over dk
 };
 
 // Each launcher returns cudaSuccess or the launch error.

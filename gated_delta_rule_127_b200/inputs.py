@@ -9,7 +9,8 @@ alpha in (0,1)^dk and a scalar write strength beta in (0,1) per token and head.
 Distributions (the same for every workload):
   q, k      ~ N(0, 1), then divided by their L2 norm per (token, head) in fp32, then cast
   v         ~ N(0, 1)
-  log_alpha = -exp(u), u ~ U(-7, -0.7)  (so log_alpha in (-0.4966, -0.00091), natural log)
+  log_alpha = -exp(u), u ~ U(-7, -0.7)  (so log_alpha in (-0.4966, -0.00091), natural log); one draw
+              per (token, head, key channel), or per (token, head) for Gated DeltaNet's scalar gate
   beta      = sigmoid(N(0, 1))
   S0        = 0.02 * N(0, 1)           (fp32; only where the workload has an initial state)
 Draw order: sequence lengths (CPU generator), then q, k, v, u, beta logits, S0.
@@ -41,7 +42,7 @@ class PrefillInputs:
     q: torch.Tensor            # [T_total, H, dk]
     k: torch.Tensor            # [T_total, H, dk]
     v: torch.Tensor            # [T_total, H, dv]
-    log_alpha: torch.Tensor    # [T_total, H, dk]
+    log_alpha: torch.Tensor    # [T_total, H, dk], or [T_total, H] with a scalar gate
     beta: torch.Tensor         # [T_total, H]
     initial_state: Optional[torch.Tensor]  # [N, H, dk, dv] fp32 or None
     cu_seqlens: torch.Tensor   # [N+1] int32 on the tensors' device
@@ -73,8 +74,9 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
 
 def make_prefill(lengths: List[int], H: int, dk: int, dv: int, *, dtype=torch.bfloat16,
                  gate_dtype=torch.float32, init_state: bool = True, seed: int = 0,
-                 device="cpu", chunk: int = 64) -> PrefillInputs:
-    """Packed variable-length prefill inputs for the given sequence lengths."""
+                 device="cpu", chunk: int = 64, scalar_gate: bool = False) -> PrefillInputs:
+    """Packed variable-length prefill inputs for the given sequence lengths (scalar_gate: one
+    log_alpha per token and head, [T, H])."""
     lengths = [int(x) for x in lengths]
     T = sum(lengths)
     g = _generator(device, seed)
@@ -82,7 +84,7 @@ def make_prefill(lengths: List[int], H: int, dk: int, dv: int, *, dtype=torch.bf
     q = _unit_rows(torch.randn((T, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
     k = _unit_rows(torch.randn((T, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
     v = torch.randn((T, H, dv), generator=g, device=device, dtype=f32).to(dtype)
-    u = torch.rand((T, H, dk), generator=g, device=device, dtype=f32) * 6.3 - 7.0
+    u = torch.rand((T, H) if scalar_gate else (T, H, dk), generator=g, device=device, dtype=f32) * 6.3 - 7.0
     log_alpha = (-torch.exp(u)).to(gate_dtype)
     del u
     beta = torch.sigmoid(torch.randn((T, H), generator=g, device=device, dtype=f32)).to(gate_dtype)
@@ -122,7 +124,7 @@ class DecodeStep:
     q: torch.Tensor          # [B, H, dk]
     k: torch.Tensor          # [B, H, dk]
     v: torch.Tensor          # [B, H, dv]
-    log_alpha: torch.Tensor  # [B, H, dk]
+    log_alpha: torch.Tensor  # [B, H, dk], or [B, H] with a scalar gate
     beta: torch.Tensor       # [B, H]
 
 
@@ -132,7 +134,7 @@ def make_decode_state(B: int, H: int, dk: int, dv: int, seed: int = 0, device="c
 
 
 def make_decode_step(step: int, B: int, H: int, dk: int, dv: int, *, dtype=torch.bfloat16,
-                     gate_dtype=torch.float32, seed: int = 0, device="cpu") -> DecodeStep:
+                     gate_dtype=torch.float32, seed: int = 0, device="cpu", scalar_gate: bool = False) -> DecodeStep:
     """Inputs of decode step `step` (0-based); each step has its own generator, seeded from
     (seed, step), so any step can be regenerated on its own."""
     g = _generator(device, seed * 1_000_003 + step + 1)
@@ -140,7 +142,7 @@ def make_decode_step(step: int, B: int, H: int, dk: int, dv: int, *, dtype=torch
     q = _unit_rows(torch.randn((B, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
     k = _unit_rows(torch.randn((B, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
     v = torch.randn((B, H, dv), generator=g, device=device, dtype=f32).to(dtype)
-    u = torch.rand((B, H, dk), generator=g, device=device, dtype=f32) * 6.3 - 7.0
+    u = torch.rand((B, H) if scalar_gate else (B, H, dk), generator=g, device=device, dtype=f32) * 6.3 - 7.0
     log_alpha = (-torch.exp(u)).to(gate_dtype)
     beta = torch.sigmoid(torch.randn((B, H), generator=g, device=device, dtype=f32)).to(gate_dtype)
     return DecodeStep(q, k, v, log_alpha, beta)

@@ -48,6 +48,10 @@ def load_library() -> ctypes.CDLL:
     lib.kda_chunk_fwd_static_scratch.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
     lib.kda_decode_step.restype = i32
+    lib.kda_gdn_chunk_fwd.argtypes = lib.kda_chunk_fwd.argtypes
+    lib.kda_gdn_chunk_fwd.restype = i32
+    lib.kda_gdn_decode_step.argtypes = lib.kda_decode_step.argtypes
+    lib.kda_gdn_decode_step.restype = i32
     lib.kda_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.kda_get_device_status.restype = i32
     lib.kda_status_string.argtypes = [i32]
@@ -124,9 +128,31 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: 
     A workspace of kda_chunk_fwd_workspace_size bytes is allocated when none is given; with
     use_workspace=False none is passed and the library runs its workspace-free kernel.
     """
+    return _chunk_fwd("kda_chunk_fwd", q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs, chunk_size,
+                      o, final_state, output_final_state, dtype_o, workspace, use_workspace, stream)
+
+
+def kda_gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                      beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
+                      cu_seqlens: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
+                      chunk_size: int = 64, o: Optional[torch.Tensor] = None,
+                      final_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
+                      dtype_o: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
+                      use_workspace: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Gated DeltaNet prefill (kda_gdn_chunk_fwd in include/kda.h): as kda_chunk_fwd with a scalar
+    log_alpha [T, H] per token and head."""
+    return _chunk_fwd("kda_gdn_chunk_fwd", q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs,
+                      chunk_size, o, final_state, output_final_state, dtype_o, workspace, use_workspace, stream)
+
+
+def _chunk_fwd(entry, q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs, chunk_size, o, final_state,
+               output_final_state, dtype_o, workspace, use_workspace, stream):
     lib = load_library()
-    if q.dim() != 3 or k.shape != q.shape or log_alpha.shape != q.shape or v.dim() != 3 or beta.dim() != 2:
-        raise ValueError("expected q, k, log_alpha [T, H, dk], v [T, H, dv], beta [T, H]")
+    scalar_gate = entry == "kda_gdn_chunk_fwd"
+    gate_shape = q.shape[:2] if scalar_gate else q.shape
+    if q.dim() != 3 or k.shape != q.shape or log_alpha.shape != gate_shape or v.dim() != 3 or beta.dim() != 2:
+        raise ValueError("expected q, k [T, H, dk], v [T, H, dv], beta [T, H], log_alpha "
+                         + ("[T, H]" if scalar_gate else "[T, H, dk]"))
     T, H, dk = q.shape
     dv = v.shape[2]
     if v.shape[:2] != (T, H) or beta.shape != (T, H):
@@ -161,12 +187,12 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: 
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(device):
-        st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
-                               _ptr(cu_seqlens), T, N, H, dk, dv, chunk_size,
-                               _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"), _dtype_code(o, "o"),
-                               _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _stream_handle(stream))
+        st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+                                 _ptr(cu_seqlens), T, N, H, dk, dv, chunk_size,
+                                 _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"), _dtype_code(o, "o"),
+                                 _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _stream_handle(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_chunk_fwd")
+        raise KdaError(st, entry)
     return o, final_state
 
 
@@ -225,9 +251,24 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha
                     dtype_o: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
     """One recurrent KDA step (see kda_decode_step in include/kda.h); `state` [B, H, dk, dv] fp32 is
     updated in place.  Returns o [B, H, dv]."""
+    return _decode("kda_decode_step", q, k, v, log_alpha, beta, state, o, dtype_o, stream)
+
+
+def kda_gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                        beta: torch.Tensor, state: torch.Tensor, *, o: Optional[torch.Tensor] = None,
+                        dtype_o: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
+    """One Gated DeltaNet step (kda_gdn_decode_step in include/kda.h): as kda_decode_step with a scalar
+    log_alpha [B, H]."""
+    return _decode("kda_gdn_decode_step", q, k, v, log_alpha, beta, state, o, dtype_o, stream)
+
+
+def _decode(entry, q, k, v, log_alpha, beta, state, o, dtype_o, stream):
     lib = load_library()
     B, H, dk = q.shape
     dv = v.shape[2]
+    gate_shape = (B, H) if entry == "kda_gdn_decode_step" else (B, H, dk)
+    if tuple(log_alpha.shape) != gate_shape:
+        raise ValueError(f"log_alpha must be {list(gate_shape)}")
     if state.dtype != torch.float32 or state.shape != (B, H, dk, dv):
         raise ValueError("state must be fp32 [B, H, dk, dv]")
     if dtype_o is None:
@@ -236,11 +277,11 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha
         o = torch.empty((B, H, dv), dtype=dtype_o, device=q.device)
     _check_cuda(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, state=state, o=o), q.device)
     with torch.cuda.device(q.device):
-        st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state), B, H, dk, dv,
+        st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state), B, H, dk, dv,
                                  _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"), _dtype_code(o, "o"),
                                  _ptr(o), _stream_handle(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_decode_step")
+        raise KdaError(st, entry)
     return o
 
 

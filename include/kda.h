@@ -157,6 +157,39 @@ KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v,
                            void* o, void* stream);
 
 /*
+ * Gated DeltaNet: the same operator with one decay rate per token and head instead of one per key
+ * channel, alpha_t = exp(log_alpha_t) a scalar in (0,1):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) alpha_t S_{t-1} + beta_t k_t v_t^T,    o_t = S_t^T q_t.
+ *
+ * Passage: "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "선형 어텐션에서
+ * Gated DeltaNet까지" (a scalar forget gate on the whole state, then the delta rule), and "From
+ * GPT-2 to Kimi K3, Explained", section "Gated DeltaNet — 망각을 더하다" (alpha = 1 is the plain
+ * delta rule, alpha = 0 clears the memory).  It is KDA with Diag(alpha_t) = alpha_t I, so these entry points run the same kernels
+ * as kda_chunk_fwd / kda_decode_step, which read the gate once per token and head and broadcast it
+ * over the dk channels.
+ *
+ * Arguments, workspace, paths, statuses and behaviour are those of kda_chunk_fwd (resp.
+ * kda_decode_step) except:
+ *   log_alpha   [T_total, H]  (resp. [B, H])  dtype_gate   natural log of the scalar decay, <= 0;
+ *               aligned to its element size (it is not read by the tensor memory copier).
+ * The workspace size is kda_chunk_fwd_workspace_size(...) of the same sizes.
+ */
+KDA_API kda_status kda_gdn_chunk_fwd(const void* q, const void* k, const void* v,
+                         const void* log_alpha, const void* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
+                         void* o, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+KDA_API kda_status kda_gdn_decode_step(const void* q, const void* k, const void* v,
+                           const void* log_alpha, const void* beta, float* state,
+                           int B, int H, int dk, int dv,
+                           kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
+                           void* o, void* stream);
+
+/*
  * Waits for `stream`, then reads and clears the sticky device flags (KDA_DEVFLAG_*) of the current
  * device into *flags (may be NULL).  Returns KDA_OK if no flag was set, KDA_ERR_TIMEOUT if the
  * timeout flag was set, KDA_ERR_DEVICE_CHECK for any other flag, KDA_ERR_CUDA on a CUDA error.

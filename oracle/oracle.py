@@ -102,3 +102,26 @@ def decode_step(q, k, v, log_alpha, beta, state, nthreads=0):
     if rc != 0:
         raise ValueError(f"kda_oracle_decode failed with code {rc}")
     return o, S
+
+
+def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, nthreads=0):
+    """Gated DeltaNet over a packed batch: log_alpha [T, H] is one decay rate per token and head.
+
+    "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "선형 어텐션에서 Gated
+    DeltaNet까지": a scalar forget gate alpha_t decays the whole state before the delta rule, which is
+    the KDA recurrence with Diag(alpha_t) = alpha_t I; the rate is repeated over the dk key channels and
+    the recurrence of ``forward`` is run.  Returns (o [T, H, dv], final_state [N, H, dk, dv]).
+    """
+    la = _f64(log_alpha)
+    T, H, dk = _f64(q).shape
+    assert la.shape == (T, H)
+    return forward(q, k, v, np.repeat(la[:, :, None], dk, axis=2), beta, initial_state, cu_seqlens,
+                   nthreads=nthreads)
+
+
+def gdn_decode_step(q, k, v, log_alpha, beta, state, nthreads=0):
+    """One Gated DeltaNet step: log_alpha [B, H], repeated over the key channels as in gdn_forward."""
+    la = _f64(log_alpha)
+    B, H, dk = _f64(q).shape
+    assert la.shape == (B, H)
+    return decode_step(q, k, v, np.repeat(la[:, :, None], dk, axis=2), beta, state, nthreads=nthreads)

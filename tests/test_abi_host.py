@@ -17,7 +17,7 @@ def lib():
 def test_header_declares_the_entry_points():
     names = set(kda.header_symbols())
     assert {"kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_get_device_status",
-            "kda_status_string", "kda_version"} <= names
+            "kda_status_string", "kda_version", "kda_gdn_chunk_fwd", "kda_gdn_decode_step"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -68,6 +68,35 @@ def _chunk(lib, **kw):
 ])
 def test_chunk_fwd_rejects_on_host(lib, kw, expect):
     assert _chunk(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(T=100, N=3), kda.KDA_ERR_INVALID_ARG),
+    (dict(la=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(la=FAKE + 2), kda.KDA_ERR_INVALID_ARG),          # [T, H] fp32 gate: needs 4-byte alignment only
+    (dict(la=FAKE + 1, dg=kda.KDA_BF16), kda.KDA_ERR_INVALID_ARG),
+    (dict(ws=FAKE, wsb=16), kda.KDA_ERR_INVALID_ARG),
+])
+def test_gdn_chunk_fwd_rejects_on_host(lib, kw, expect):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, cu=None, T=128, N=1, H=2, dk=128, dv=128,
+             chunk=64, dq=kda.KDA_BF16, dg=kda.KDA_FP32, do=kda.KDA_FP32, o=FAKE, sf=None, ws=None, wsb=0)
+    a.update(kw)
+    st = lib.kda_gdn_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["cu"], a["T"], a["N"],
+                               a["H"], a["dk"], a["dv"], a["chunk"], a["dq"], a["dg"], a["do"], a["o"], a["sf"],
+                               a["ws"], a["wsb"], None)
+    assert st == expect
+
+
+def test_gdn_decode_step_rejects_on_host(lib):
+    args = lambda **kw: [kw.get(n, d) for n, d in [("q", FAKE), ("k", FAKE), ("v", FAKE), ("la", FAKE),
+                                                   ("beta", FAKE), ("S", FAKE), ("B", 4), ("H", 2), ("dk", 128),
+                                                   ("dv", 128), ("dq", kda.KDA_BF16), ("dg", kda.KDA_FP32),
+                                                   ("do", kda.KDA_FP32), ("o", FAKE)]] + [None]
+    assert lib.kda_gdn_decode_step(*args(la=FAKE + 2)) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_gdn_decode_step(*args(dk=32)) == kda.KDA_ERR_UNSUPPORTED
+    assert lib.kda_gdn_decode_step(*args(B=0)) == kda.KDA_OK
 
 
 def _decode(lib, **kw):

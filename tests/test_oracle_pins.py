@@ -121,6 +121,32 @@ def test_scalar_alpha_reduces_to_gated_deltanet(fwd=oracle.forward):
     np.testing.assert_allclose(sf[0], gamma[-1][:, None, None] * sf_dn[0], rtol=1e-9, atol=1e-12)
 
 
+def test_gdn_entry_points_follow_the_textbook_recurrence():
+    """oracle.gdn_forward / gdn_decode_step (scalar log_alpha [T, H]) against the separately written
+    Gated DeltaNet recurrence, over two packed sequences; and the decode step against one
+    textbook step."""
+    rng = np.random.default_rng(13)
+    T, H, dk, dv = 30, 2, 6, 3
+    q, k, v, _, beta, _ = _rand_inputs(rng, T, H, dk, dv)
+    a_scalar = -np.exp(rng.uniform(-4.0, -0.5, (T, H)))
+    s0 = 0.3 * rng.standard_normal((2, H, dk, dv))
+    cu = np.array([0, 11, T])
+    o, sf = oracle.gdn_forward(q, k, v, a_scalar, beta, s0, cu)
+    for n in range(2):
+        a, b = cu[n], cu[n + 1]
+        for h in range(H):
+            o_ref, s_ref = _gdn_textbook(q[a:b, h], k[a:b, h], v[a:b, h], np.exp(a_scalar[a:b, h]), beta[a:b, h],
+                                         s0[n, h])
+            np.testing.assert_allclose(o[a:b, h], o_ref, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(sf[n, h], s_ref, rtol=1e-12, atol=1e-12)
+    od, Sd = oracle.gdn_decode_step(q[:1].reshape(1, H, dk), k[:1].reshape(1, H, dk), v[:1].reshape(1, H, dv),
+                                    a_scalar[:1], beta[:1], s0[:1])
+    for h in range(H):
+        o_ref, s_ref = _gdn_textbook(q[:1, h], k[:1, h], v[:1, h], np.exp(a_scalar[:1, h]), beta[:1, h], s0[0, h])
+        np.testing.assert_allclose(od[0, h], o_ref[0], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(Sd[0, h], s_ref, rtol=1e-12, atol=1e-12)
+
+
 def test_write_read_invariant(fwd=oracle.forward):
     """With ||k_t|| = 1 and beta_t = 1 the state returns v_t for key k_t right after the write."""
     rng = np.random.default_rng(4)
