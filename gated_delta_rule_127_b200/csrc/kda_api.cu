@@ -43,11 +43,15 @@ bool supported_dim(int d) { return d == 64 || d == 128; }
 
 }  // namespace
 
-// kda_chunk_fwd and kda_gdn_chunk_fwd: scalar_gate selects a [T_total, H] log_alpha.
+constexpr uint32_t kKnownOptions = KDA_OPT_SCALAR_GATE | KDA_OPT_L2NORM_QK | KDA_OPT_BETA_LOGITS;
+
+// kda_chunk_fwd, kda_gdn_chunk_fwd and kda_chunk_fwd_ex (KDA_OPT_* options).
 kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                      const float* initial_state, const int32_t* cu_seqlens, int64_t T_total, int N, int H, int dk,
                      int dv, int chunk_size, kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
-                     float* final_state, void* workspace, size_t workspace_bytes, void* stream, bool scalar_gate) {
+                     float* final_state, void* workspace, size_t workspace_bytes, void* stream, uint32_t options) {
+    const bool scalar_gate = (options & KDA_OPT_SCALAR_GATE) != 0;
+    if (options & ~kKnownOptions) return KDA_ERR_INVALID_ARG;
     if (T_total < 0 || N <= 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk_size <= 0)
         return KDA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
@@ -77,6 +81,8 @@ kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* lo
     a.o = o; a.final_state = final_state; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     a.stream = static_cast<cudaStream_t>(stream);
     a.scalar_gate = scalar_gate;
+    a.l2norm_qk = (options & KDA_OPT_L2NORM_QK) != 0;
+    a.beta_logits = (options & KDA_OPT_BETA_LOGITS) != 0;
     if (device_flags_ptr(&a.flags) != cudaSuccess) return KDA_ERR_CUDA;
 
     cudaError_t err;
@@ -91,10 +97,12 @@ kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* lo
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-// kda_decode_step and kda_gdn_decode_step: scalar_gate selects a [B, H] log_alpha.
+// kda_decode_step, kda_gdn_decode_step and kda_decode_step_ex (KDA_OPT_* options).
 kda_status decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                        float* state, int B, int H, int dk, int dv, kda_dtype dtype_qkv, kda_dtype dtype_gate,
-                       kda_dtype dtype_o, void* o, void* stream, bool scalar_gate) {
+                       kda_dtype dtype_o, void* o, void* stream, uint32_t options) {
+    const bool scalar_gate = (options & KDA_OPT_SCALAR_GATE) != 0;
+    if (options & ~kKnownOptions) return KDA_ERR_INVALID_ARG;
     if (B < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
         return KDA_ERR_INVALID_ARG;
@@ -114,6 +122,8 @@ kda_status decode_step(const void* q, const void* k, const void* v, const void* 
     a.stream = static_cast<cudaStream_t>(stream);
     a.flags = nullptr;
     a.scalar_gate = scalar_gate;
+    a.l2norm_qk = (options & KDA_OPT_L2NORM_QK) != 0;
+    a.beta_logits = (options & KDA_OPT_BETA_LOGITS) != 0;
     return launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -133,7 +143,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                          kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
                          float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
     return kda::chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, T_total, N, H, dk, dv, chunk_size,
-                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, false);
+                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, 0u);
 }
 
 kda_status kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
@@ -142,7 +152,7 @@ kda_status kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const 
                              kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
                              float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
     return kda::chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, T_total, N, H, dk, dv, chunk_size,
-                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, true);
+                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, KDA_OPT_SCALAR_GATE);
 }
 
 kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
@@ -150,7 +160,7 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const vo
                            kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
                            void* stream) {
     return kda::decode_step(q, k, v, log_alpha, beta, state, B, H, dk, dv, dtype_qkv, dtype_gate, dtype_o, o,
-                            stream, false);
+                            stream, 0u);
 }
 
 kda_status kda_gdn_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
@@ -158,7 +168,25 @@ kda_status kda_gdn_decode_step(const void* q, const void* k, const void* v, cons
                                kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
                                void* stream) {
     return kda::decode_step(q, k, v, log_alpha, beta, state, B, H, dk, dv, dtype_qkv, dtype_gate, dtype_o, o,
-                            stream, true);
+                            stream, KDA_OPT_SCALAR_GATE);
+}
+
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha,
+                            const void* beta, const float* initial_state, const int32_t* cu_seqlens,
+                            int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                            kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                            float* final_state, void* workspace, size_t workspace_bytes, uint32_t options,
+                            void* stream) {
+    return kda::chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, T_total, N, H, dk, dv, chunk_size,
+                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, options);
+}
+
+kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const void* log_alpha,
+                              const void* beta, float* state, int B, int H, int dk, int dv,
+                              kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
+                              uint32_t options, void* stream) {
+    return kda::decode_step(q, k, v, log_alpha, beta, state, B, H, dk, dv, dtype_qkv, dtype_gate, dtype_o, o,
+                            stream, options);
 }
 
 kda_status kda_get_device_status(void* stream, uint32_t* flags) {

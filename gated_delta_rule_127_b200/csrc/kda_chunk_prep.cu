@@ -65,7 +65,8 @@ constexpr uint32_t OFF_X = 217600;     // 32 x 32 fp32 scratch for the inverse
 constexpr uint32_t OFF_TASK = 221696;  // three Task slots (this task, the next, the one after)
 constexpr uint32_t OFF_BARS = 221792;  // mbarriers: TMA, MMAs 1-2, MMAs 3-4, MMAs 5-6; then the TMEM base address
 constexpr uint32_t OFF_SAL = 221840;   // scalar log-decay [2][64] (Gated DeltaNet gates), by task parity
-constexpr uint32_t SMEM_USED = OFF_SAL + 512;
+constexpr uint32_t OFF_RN = OFF_SAL + 512;  // 1 / ||k_r|| [64], 1 / ||q_r|| [64] (fused L2 normalisation)
+constexpr uint32_t SMEM_USED = OFF_RN + 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 // after MMA 1 (k, v staging and K- are dead):
 constexpr uint32_t OFF_A = 49152;      // A fp32 [64][TP]
@@ -280,13 +281,14 @@ __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, f
 
 // SG: Gated DeltaNet gates -- log_alpha is [T_total, H], one decay rate per token and head, read
 // with beta and broadcast over the key channels (tm_g is then unused).
-template <typename TG, bool SG>
+// PRO: q and k arrive raw; every use of a row is scaled by 1 / its L2 norm, computed per chunk.
+template <typename TG, bool SG, bool PRO>
 __global__ void __launch_bounds__(THREADS, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const TG* __restrict__ beta, const TG* __restrict__ log_alpha_sg,
                   const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H,
-                  unsigned char* __restrict__ ws, unsigned int* flags) {
+                  unsigned char* __restrict__ ws, unsigned int* flags, int beta_logits) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;   // tensor-memory lane quadrant
     const int qr = warp >> 2;  // row quarter (elementwise pass) / column quarter (read-outs)
@@ -302,6 +304,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float* x_egm = x_gc + 128;
     float* x_gam = x_egm + 128;
     float* s_alpha2 = reinterpret_cast<float*>(sm + OFF_SAL);  // [2][64] (SG only)
+    float* s_rn = reinterpret_cast<float*>(sm + OFF_RN);       // [128]: k rows, then q rows (PRO only)
     float* xs = reinterpret_cast<float*>(sm + OFF_X);
     Task* slots = reinterpret_cast<Task*>(sm + OFF_TASK);  // ring of 3: this task, the next, the one after
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
@@ -359,7 +362,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto load_beta = [&](const Task& t, uint32_t parity) {
         const int r = tid - 64;
         if (r >= 0 && r < C && t.id >= 0)
-            s_beta2[64 * parity + r] = r < t.len ? to_f32(beta[(t.c0 + r) * H + t.h]) : 0.f;
+            s_beta2[64 * parity + r] = r < t.len ? beta_value(to_f32(beta[(t.c0 + r) * H + t.h]), beta_logits) : 0.f;
         if (SG && tid < C && t.id >= 0)
             s_alpha2[64 * parity + tid] = tid < t.len ? to_f32(log_alpha_sg[(t.c0 + tid) * H + t.h]) : 0.f;
     };
@@ -389,6 +392,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             x_part[qr * 128 + c] = run;
         }
+        if (PRO) {  // 1 / ||k_r|| and 1 / ||q_r||: warp w takes rows 8 w .. 8 w + 7 of [K; Q], 4 channels a lane
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int row = 8 * warp + j, r = row & 63;
+                const uint2 u = *reinterpret_cast<const uint2*>(sm + (row < 64 ? OFF_SK : OFF_SQ) + bf16_sw_off(r, 4 * lane));
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+                float ss = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                if (lane == 0) s_rn[row] = inv_norm(ss);
+            }
+        }
         __syncthreads();
         {
             float off = 0.f;
@@ -414,7 +430,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int u = 0; u < 4; ++u) {
                     const int R = rb + r4 + u;
                     const bool live = R < len;
-                    const float kv = live ? __bfloat162float(sk[bf16_sw_off(R, c) >> 1]) : 0.f;
+                    const float kv = live ? __bfloat162float(sk[bf16_sw_off(R, c) >> 1]) * (PRO ? s_rn[R] : 1.f) : 0.f;
                     const float vv = live ? __bfloat162float(sv[bf16_sw_off(R, c) >> 1]) : 0.f;
                     const float b = s_beta[R];
                     const float e = __expf(g[r4 + u] - gm), ie = __expf(gm - g[r4 + u]);
@@ -439,6 +455,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const unsigned char* src = sm + (c < 64 ? OFF_SK : OFF_SQ);
             const bool live = r < len;
             const int cb = 32 * qr;
+            const float rn = PRO ? s_rn[c] : 1.f;  // lanes 0..63 k rows, 64..127 q rows
             float v[32];
 #pragma unroll
             for (int e8 = 0; e8 < 4; ++e8) {
@@ -449,7 +466,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const float4 e1 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(r, cc + 4, 64));
                 const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[8 * e8 + i] = live ? to_tf32(x[i] * ev[i]) : 0.f;
+                for (int i = 0; i < 8; ++i) v[8 * e8 + i] = live ? to_tf32(x[i] * rn * ev[i]) : 0.f;
             }
             tmem_st32(tq + TM_A1 + cb, v);
             tmem_st_wait();
@@ -604,6 +621,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // K-major rows t
             const int t = 16 * q4 + (lane & 15), hc = lane >> 4;
             const bool live = t < len;
+            const float rq = PRO ? s_rn[64 + t] : 1.f;
             float x[16];
             tmem_ld16_x2<16>(tq + TM_PW + 32 * qr, x);
             unsigned char* row = sm + STG_Q + qr * 8192 + t * 128;  // K-block qr, row t
@@ -618,7 +636,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float qh[8];
 #pragma unroll
                 for (int w = 0; w < 8; ++w)
-                    qh[w] = to_tf32((live ? qv[w] * ev[w] * x_egm[cc + w] : 0.f) - x[8 * e8 + w]);
+                    qh[w] = to_tf32((live ? qv[w] * rq * ev[w] * x_egm[cc + w] : 0.f) - x[8 * e8 + w]);
                 const int ch = 4 * hc + 2 * e8;  // 16-byte chunk of the row within the K-block
                 *reinterpret_cast<float4*>(row + ((ch ^ (t & 7)) << 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
                 *reinterpret_cast<float4*>(row + (((ch + 1) ^ (t & 7)) << 4)) = make_float4(qh[4], qh[5], qh[6], qh[7]);
@@ -678,7 +696,7 @@ int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <typename TG, bool SG>
+template <typename TG, bool SG, bool PRO>
 cudaError_t launch_prep(const ChunkArgs& a) {
     CUtensorMap mq, mk, mv, mg;
     const uint64_t T = static_cast<uint64_t>(a.T_total), H = static_cast<uint64_t>(a.H);
@@ -693,7 +711,7 @@ cudaError_t launch_prep(const ChunkArgs& a) {
         (!SG && !tma_encode_blocks(&mg, a.log_alpha, gdt, sizeof(TG), DK, H, T, gblk, C, sw)))
         return cudaErrorInvalidValue;
     if (SG) mg = mq;  // not read
-    auto kern = chunk_prep_kernel<TG, SG>;
+    auto kern = chunk_prep_kernel<TG, SG, PRO>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int64_t ntasks = wy::num_slots(a.T_total, a.N) * a.H;
@@ -702,7 +720,7 @@ cudaError_t launch_prep(const ChunkArgs& a) {
     kern<<<grid, THREADS, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, static_cast<const TG*>(a.beta),
                                                   SG ? static_cast<const TG*>(a.log_alpha) : nullptr, a.cu_seqlens,
                                                   a.T_total, a.N, a.H, static_cast<unsigned char*>(a.workspace),
-                                                  a.flags);
+                                                  a.flags, a.beta_logits ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -713,9 +731,14 @@ size_t chunk_wy_workspace_size(int64_t T_total, int N, int H, int dk, int dv) {
     return static_cast<size_t>(wy::num_slots(T_total, N)) * static_cast<size_t>(H) * wy::REC_BYTES;
 }
 
+template <bool SG>
+cudaError_t launch_prep_sg(const ChunkArgs& a) {
+    if (a.l2norm_qk) return a.dtype_gate == KDA_FP32 ? launch_prep<float, SG, true>(a) : launch_prep<__nv_bfloat16, SG, true>(a);
+    return a.dtype_gate == KDA_FP32 ? launch_prep<float, SG, false>(a) : launch_prep<__nv_bfloat16, SG, false>(a);
+}
+
 cudaError_t launch_chunk_prep(const ChunkArgs& a) {
-    if (a.scalar_gate) return a.dtype_gate == KDA_FP32 ? launch_prep<float, true>(a) : launch_prep<__nv_bfloat16, true>(a);
-    return a.dtype_gate == KDA_FP32 ? launch_prep<float, false>(a) : launch_prep<__nv_bfloat16, false>(a);
+    return a.scalar_gate ? launch_prep_sg<true>(a) : launch_prep_sg<false>(a);
 }
 
 }  // namespace kda

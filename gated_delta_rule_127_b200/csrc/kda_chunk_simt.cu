@@ -100,7 +100,7 @@ chunk_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
                   const TG* __restrict__ log_alpha, const TG* __restrict__ beta,
                   const float* initial_state, const int32_t* __restrict__ cu_seqlens,
                   int64_t T_total, int N, int H, int DV, TO* __restrict__ o, float* final_state,
-                  unsigned int* flags, int scalar_gate) {
+                  unsigned int* flags, int scalar_gate, int l2norm_qk, int beta_logits) {
     using Sm = SimtSmem<DK>;
     constexpr int KP = Sm::KP;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -156,9 +156,21 @@ chunk_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
             const int r = idx / DVS, j = idx % DVS;
             s.vr[idx] = r < len ? to_f32(v[(c0 + r) * v_row + (int64_t)h * DV + col0 + j]) : 0.f;
         }
-        if (tid < C) s.beta[tid] = tid < len ? to_f32(beta[(c0 + tid) * H + h]) : 0.f;
+        if (tid < C) s.beta[tid] = tid < len ? beta_value(to_f32(beta[(c0 + tid) * H + h]), beta_logits != 0) : 0.f;
         if (tid == 0) s.exact = 0;
         __syncthreads();
+        if (l2norm_qk) {  // fused L2 normalisation of the chunk's k and q rows, in place, one warp per row
+            for (int row = warp; row < 2 * C; row += THREADS / 32) {
+                float* x = (row < C ? s.kx : s.qx) + (row % C) * KP;
+                float ss = 0.f;
+                for (int c = lane; c < DK; c += 32) ss += x[c] * x[c];
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                const float f = inv_norm(ss);
+                for (int c = lane; c < DK; c += 32) x[c] *= f;
+            }
+            __syncthreads();
+        }
         // ---- g = cumulative log-decay along the chunk, per key channel
         for (int c = tid; c < DK; c += THREADS) {
             float run = 0.f;
@@ -301,7 +313,7 @@ cudaError_t launch_typed(const ChunkArgs& a) {
         static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.v),
         static_cast<const TG*>(a.log_alpha), static_cast<const TG*>(a.beta), a.initial_state,
         a.cu_seqlens, a.T_total, a.N, a.H, a.dv, static_cast<TO*>(a.o), a.final_state, a.flags,
-        a.scalar_gate ? 1 : 0);
+        a.scalar_gate ? 1 : 0, a.l2norm_qk ? 1 : 0, a.beta_logits ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -86,7 +86,8 @@ constexpr uint32_t OFF_BAR = 228608;   // mbarrier: MMA completion
 constexpr uint32_t OFF_TBAR = 228616;  // mbarrier: TMA completion
 constexpr uint32_t OFF_SLOT = 228624;  // tensor-memory base address
 constexpr uint32_t OFF_BAR2 = 228632;  // mbarrier: completion of the second half of MMA batch 1
-constexpr uint32_t SMEM_USED = 228640;
+constexpr uint32_t OFF_RN = 228640;    // 1 / ||k_r|| [64], 1 / ||q_r|| [64] (fused L2 normalisation)
+constexpr uint32_t SMEM_USED = OFF_RN + 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 
 // Tensor-memory columns (fp32).  Batch 2 writes Y into the columns Z was read from.
@@ -204,14 +205,15 @@ __device__ __forceinline__ void store_row8<__nv_bfloat16>(__nv_bfloat16* dst, co
 
 // SG: Gated DeltaNet gates -- log_alpha is [T_total, H], one decay rate per token and head, read
 // with beta and broadcast over the key channels (tm_la is then unused).
-template <typename TG, bool SG>
+// PRO: q and k arrive raw; every use of a row is scaled by 1 / its L2 norm, computed per chunk.
+template <typename TG, bool SG, bool PRO>
 __global__ void __launch_bounds__(THREADS, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
                 const TG* __restrict__ beta, const TG* __restrict__ log_alpha_sg,
                 const float* initial_state, const int32_t* __restrict__ cu_seqlens,
                 int64_t T_total, int N, int H, void* __restrict__ o_ptr, int o_is_f32, float* final_state,
-                unsigned int* flags) {
+                unsigned int* flags, int beta_logits) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -292,7 +294,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int j = 0; j < 8; ++j) S[j] = 0.f;
     }
     float beta_next = 0.f, alpha_next = 0.f;  // alpha_next: SG only
-    if (tid < C && t0 + tid < t1) beta_next = to_f32(beta[(t0 + tid) * H + h]);
+    if (tid < C && t0 + tid < t1) beta_next = beta_value(to_f32(beta[(t0 + tid) * H + h]), beta_logits);
     if (SG && tid < C && t0 + tid < t1) alpha_next = to_f32(log_alpha_sg[(t0 + tid) * H + h]);
 
     // Matrix descriptors at K-step 0; K-step kk adds its byte offset >> 4 to the start-address field.
@@ -329,6 +331,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             x_part[qr * 128 + c] = run;
         }
+        if (PRO) {  // 1 / ||k_r|| and 1 / ||q_r||: warp w takes rows 8 w .. 8 w + 7 of [K; Q], 4 channels a lane
+            float* s_rn = tile(sm, OFF_RN);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int row = 8 * warp + j, r = row & 63;
+                const __nv_bfloat16* src = row < 64 ? sk : sq;
+                const uint2 u = *reinterpret_cast<const uint2*>(src + r * DK + 4 * lane);
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+                float ss = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                if (lane == 0) s_rn[row] = inv_norm(ss);
+            }
+        }
         __syncthreads();
         {
             float off = 0.f;
@@ -352,8 +369,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int u = 0; u < 4; ++u) {
                 const int r = rb + r4 + u;
                 const bool live = r < len;
-                const float kv = live ? __bfloat162float(sk[r * DK + c]) : 0.f;
-                const float qv = live ? __bfloat162float(sq[r * DK + c]) : 0.f;
+                const float kv = live ? __bfloat162float(sk[r * DK + c]) * (PRO ? tile(sm, OFF_RN)[r] : 1.f) : 0.f;
+                const float qv = live ? __bfloat162float(sq[r * DK + c]) * (PRO ? tile(sm, OFF_RN)[64 + r] : 1.f) : 0.f;
                 const float e = __expf(g[r4 + u] - gm), ie = __expf(gm - g[r4 + u]);
                 kp[u] = to_tf32(kv * e);
                 qp[u] = to_tf32(qv * e);
@@ -396,7 +413,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_3d(sm + OFF_SV, &tm_v, col0, h, static_cast<int>(c1), tbar);
         }
         tma_pending = c1 < t1;
-        if (tid < C) beta_next = (c1 + tid < t1) ? to_f32(beta[(c1 + tid) * H + h]) : 0.f;
+        if (tid < C) beta_next = (c1 + tid < t1) ? beta_value(to_f32(beta[(c1 + tid) * H + h]), beta_logits) : 0.f;
         if (SG && tid < C) alpha_next = (c1 + tid < t1) ? to_f32(log_alpha_sg[(c1 + tid) * H + h]) : 0.f;
 
         // ---- MMA batch 1: [A_raw; P] = [K+; Q+] (K-)^T,  Z = K+ S',  O = Q+ S'
@@ -548,7 +565,7 @@ bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TG, bool SG>
+template <typename TG, bool SG, bool PRO>
 cudaError_t launch_typed(const ChunkArgs& a) {
     CUtensorMap mq, mk, mla, mv;
     const uint64_t T = static_cast<uint64_t>(a.T_total), H = static_cast<uint64_t>(a.H);
@@ -559,14 +576,14 @@ cudaError_t launch_typed(const ChunkArgs& a) {
         !encode_3d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, H, T, DVS, C))
         return cudaErrorInvalidValue;
     if (SG) mla = mq;  // not read
-    auto kern = chunk_tc_kernel<TG, SG>;
+    auto kern = chunk_tc_kernel<TG, SG, PRO>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int64_t blocks = static_cast<int64_t>(a.N) * a.H * (DV / DVS);
     kern<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
         mq, mk, mla, mv, static_cast<const TG*>(a.beta), SG ? static_cast<const TG*>(a.log_alpha) : nullptr,
         a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
-        a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags);
+        a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags, a.beta_logits ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -577,9 +594,14 @@ bool chunk_tc_supported(const ChunkArgs& a) {
     return a.dtype_qkv == KDA_BF16 && a.dk == DK && a.dv == DV && a.T_total > 0 && a.T_total < (int64_t(1) << 31);
 }
 
+template <bool SG>
+cudaError_t launch_sg(const ChunkArgs& a) {
+    if (a.l2norm_qk) return a.dtype_gate == KDA_FP32 ? launch_typed<float, SG, true>(a) : launch_typed<__nv_bfloat16, SG, true>(a);
+    return a.dtype_gate == KDA_FP32 ? launch_typed<float, SG, false>(a) : launch_typed<__nv_bfloat16, SG, false>(a);
+}
+
 cudaError_t launch_chunk_tc(const ChunkArgs& a) {
-    if (a.scalar_gate) return a.dtype_gate == KDA_FP32 ? launch_typed<float, true>(a) : launch_typed<__nv_bfloat16, true>(a);
-    return a.dtype_gate == KDA_FP32 ? launch_typed<float, false>(a) : launch_typed<__nv_bfloat16, false>(a);
+    return a.scalar_gate ? launch_sg<true>(a) : launch_sg<false>(a);
 }
 
 

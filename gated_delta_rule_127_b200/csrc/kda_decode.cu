@@ -29,7 +29,8 @@ template <int DK, int DV, typename TIn, typename TG, typename TO>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, 2)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                    const TG* __restrict__ log_alpha, const TG* __restrict__ beta,
-                   float* __restrict__ state, TO* __restrict__ o, int scalar_gate) {
+                   float* __restrict__ state, TO* __restrict__ o, int scalar_gate, int l2norm_qk,
+                   int beta_logits) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int TPR = Sh::TPR, RG = Sh::RG, RPT = Sh::RPT;
 
@@ -56,8 +57,22 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
         s_alpha[c] = expf(to_f32(log_alpha[scalar_gate ? u : u * DK + c]));  // GDN: one rate per (b, h)
     }
     for (int j = tid; j < DV; j += Sh::THREADS) s_v[j] = to_f32(v[u * DV + j]);
-    const float b = to_f32(beta[u]);
+    const float b = beta_value(to_f32(beta[u]), beta_logits != 0);
     __syncthreads();
+    if (l2norm_qk) {  // fused L2 normalisation of k and q, in place (warp 0)
+        if (tid < 32) {
+            float sk = 0.f, sq = 0.f;
+            for (int c = tid; c < DK; c += 32) { sk += s_k[c] * s_k[c]; sq += s_q[c] * s_q[c]; }
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, m);
+                sq += __shfl_xor_sync(0xffffffffu, sq, m);
+            }
+            const float fk = inv_norm(sk), fq = inv_norm(sq);
+            for (int c = tid; c < DK; c += 32) { s_k[c] *= fk; s_q[c] *= fq; }
+        }
+        __syncthreads();
+    }
 
     if (tid < 32) {  // k^T q, needed for the output only
         float acc = 0.f;
@@ -106,7 +121,7 @@ cudaError_t launch_typed(const DecodeArgs& a) {
     decode_step_kernel<DK, DV, TIn, TG, TO><<<a.B * a.H, Sh::THREADS, 0, a.stream>>>(
         static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.v),
         static_cast<const TG*>(a.log_alpha), static_cast<const TG*>(a.beta), a.state,
-        static_cast<TO*>(a.o), a.scalar_gate ? 1 : 0);
+        static_cast<TO*>(a.o), a.scalar_gate ? 1 : 0, a.l2norm_qk ? 1 : 0, a.beta_logits ? 1 : 0);
     return cudaGetLastError();
 }
 

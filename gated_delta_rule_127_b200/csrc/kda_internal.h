@@ -26,6 +26,8 @@ struct ChunkArgs {
     unsigned int* flags;  // device address of the sticky flag word
     cudaStream_t stream;
     bool scalar_gate;     // log_alpha is [T_total, H] (Gated DeltaNet), broadcast over dk
+    bool l2norm_qk;       // q, k raw: divided by their L2 norm per (token, head) in the kernels
+    bool beta_logits;     // beta holds logits: sigmoid applied in the kernels
 };
 
 struct DecodeArgs {
@@ -41,6 +43,8 @@ struct DecodeArgs {
     unsigned int* flags;
     cudaStream_t stream;
     bool scalar_gate;  // log_alpha is [B, H] (Gated DeltaNet), broadcast over dk
+    bool l2norm_qk;    // q, k raw: divided by their L2 norm per (b, h) in the kernel
+    bool beta_logits;  // beta holds logits: sigmoid applied in the kernel
 };
 
 // Each launcher returns cudaSuccess or the launch error.

@@ -14,6 +14,8 @@ Distributions (the same for every workload):
   beta      = sigmoid(N(0, 1))
   S0        = 0.02 * N(0, 1)           (fp32; only where the workload has an initial state)
 Draw order: sequence lengths (CPU generator), then q, k, v, u, beta logits, S0.
+With raw=True (inputs of the fused prologue) q and k are left unnormalised and beta is returned as
+its logits; every number drawn is the same.
 """
 from dataclasses import dataclass
 from typing import List, Optional
@@ -74,20 +76,22 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
 
 def make_prefill(lengths: List[int], H: int, dk: int, dv: int, *, dtype=torch.bfloat16,
                  gate_dtype=torch.float32, init_state: bool = True, seed: int = 0,
-                 device="cpu", chunk: int = 64, scalar_gate: bool = False) -> PrefillInputs:
+                 device="cpu", chunk: int = 64, scalar_gate: bool = False, raw: bool = False) -> PrefillInputs:
     """Packed variable-length prefill inputs for the given sequence lengths (scalar_gate: one
-    log_alpha per token and head, [T, H])."""
+    log_alpha per token and head, [T, H]; raw: q, k unnormalised and beta as logits)."""
+    unit = (lambda x: x) if raw else _unit_rows
+    squash = (lambda x: x) if raw else torch.sigmoid
     lengths = [int(x) for x in lengths]
     T = sum(lengths)
     g = _generator(device, seed)
     f32 = torch.float32
-    q = _unit_rows(torch.randn((T, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
-    k = _unit_rows(torch.randn((T, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
+    q = unit(torch.randn((T, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
+    k = unit(torch.randn((T, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
     v = torch.randn((T, H, dv), generator=g, device=device, dtype=f32).to(dtype)
     u = torch.rand((T, H) if scalar_gate else (T, H, dk), generator=g, device=device, dtype=f32) * 6.3 - 7.0
     log_alpha = (-torch.exp(u)).to(gate_dtype)
     del u
-    beta = torch.sigmoid(torch.randn((T, H), generator=g, device=device, dtype=f32)).to(gate_dtype)
+    beta = squash(torch.randn((T, H), generator=g, device=device, dtype=f32)).to(gate_dtype)
     s0 = None
     if init_state:
         s0 = 0.02 * torch.randn((len(lengths), H, dk, dv), generator=g, device=device, dtype=f32)
@@ -134,15 +138,18 @@ def make_decode_state(B: int, H: int, dk: int, dv: int, seed: int = 0, device="c
 
 
 def make_decode_step(step: int, B: int, H: int, dk: int, dv: int, *, dtype=torch.bfloat16,
-                     gate_dtype=torch.float32, seed: int = 0, device="cpu", scalar_gate: bool = False) -> DecodeStep:
+                     gate_dtype=torch.float32, seed: int = 0, device="cpu", scalar_gate: bool = False,
+                     raw: bool = False) -> DecodeStep:
     """Inputs of decode step `step` (0-based); each step has its own generator, seeded from
     (seed, step), so any step can be regenerated on its own."""
     g = _generator(device, seed * 1_000_003 + step + 1)
     f32 = torch.float32
-    q = _unit_rows(torch.randn((B, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
-    k = _unit_rows(torch.randn((B, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
+    unit = (lambda x: x) if raw else _unit_rows
+    q = unit(torch.randn((B, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
+    k = unit(torch.randn((B, H, dk), generator=g, device=device, dtype=f32)).to(dtype)
     v = torch.randn((B, H, dv), generator=g, device=device, dtype=f32).to(dtype)
     u = torch.rand((B, H) if scalar_gate else (B, H, dk), generator=g, device=device, dtype=f32) * 6.3 - 7.0
     log_alpha = (-torch.exp(u)).to(gate_dtype)
-    beta = torch.sigmoid(torch.randn((B, H), generator=g, device=device, dtype=f32)).to(gate_dtype)
+    beta = torch.randn((B, H), generator=g, device=device, dtype=f32)
+    beta = (beta if raw else torch.sigmoid(beta)).to(gate_dtype)
     return DecodeStep(q, k, v, log_alpha, beta)

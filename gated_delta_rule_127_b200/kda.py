@@ -19,6 +19,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "kda.h")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_DEVICE_CHECK = range(6)
 KDA_BF16, KDA_FP32 = 0, 1
 KDA_DEVFLAG_CU_SEQLENS, KDA_DEVFLAG_DECAY_RANGE, KDA_DEVFLAG_TIMEOUT = 0x1, 0x2, 0x4
+KDA_OPT_SCALAR_GATE, KDA_OPT_L2NORM_QK, KDA_OPT_BETA_LOGITS = 0x1, 0x2, 0x4
 
 _lib = None
 
@@ -52,6 +53,10 @@ def load_library() -> ctypes.CDLL:
     lib.kda_gdn_chunk_fwd.restype = i32
     lib.kda_gdn_decode_step.argtypes = lib.kda_decode_step.argtypes
     lib.kda_gdn_decode_step.restype = i32
+    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-1] + [ctypes.c_uint32, vp]
+    lib.kda_chunk_fwd_ex.restype = i32
+    lib.kda_decode_step_ex.argtypes = lib.kda_decode_step.argtypes[:-1] + [ctypes.c_uint32, vp]
+    lib.kda_decode_step_ex.restype = i32
     lib.kda_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.kda_get_device_status.restype = i32
     lib.kda_status_string.argtypes = [i32]
@@ -145,10 +150,24 @@ def kda_gdn_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alp
                       chunk_size, o, final_state, output_final_state, dtype_o, workspace, use_workspace, stream)
 
 
+def kda_chunk_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                     beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
+                     cu_seqlens: Optional[torch.Tensor] = None, *, options: int = 0, num_seqs: Optional[int] = None,
+                     chunk_size: int = 64, o: Optional[torch.Tensor] = None,
+                     final_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
+                     dtype_o: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
+                     use_workspace: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kda_chunk_fwd_ex (include/kda.h): kda_chunk_fwd with KDA_OPT_* options (scalar gate, fused L2
+    normalisation of q and k, beta given as logits)."""
+    return _chunk_fwd("kda_chunk_fwd_ex", q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs,
+                      chunk_size, o, final_state, output_final_state, dtype_o, workspace, use_workspace, stream,
+                      options)
+
+
 def _chunk_fwd(entry, q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs, chunk_size, o, final_state,
-               output_final_state, dtype_o, workspace, use_workspace, stream):
+               output_final_state, dtype_o, workspace, use_workspace, stream, options=0):
     lib = load_library()
-    scalar_gate = entry == "kda_gdn_chunk_fwd"
+    scalar_gate = entry == "kda_gdn_chunk_fwd" or bool(options & KDA_OPT_SCALAR_GATE)
     gate_shape = q.shape[:2] if scalar_gate else q.shape
     if q.dim() != 3 or k.shape != q.shape or log_alpha.shape != gate_shape or v.dim() != 3 or beta.dim() != 2:
         raise ValueError("expected q, k [T, H, dk], v [T, H, dv], beta [T, H], log_alpha "
@@ -187,10 +206,12 @@ def _chunk_fwd(entry, q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_s
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(device):
+        extra = (int(options),) if entry == "kda_chunk_fwd_ex" else ()
         st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
                                  _ptr(cu_seqlens), T, N, H, dk, dv, chunk_size,
                                  _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"), _dtype_code(o, "o"),
-                                 _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _stream_handle(stream))
+                                 _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, *extra,
+                                 _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, entry)
     return o, final_state
@@ -262,11 +283,19 @@ def kda_gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a
     return _decode("kda_gdn_decode_step", q, k, v, log_alpha, beta, state, o, dtype_o, stream)
 
 
-def _decode(entry, q, k, v, log_alpha, beta, state, o, dtype_o, stream):
+def kda_decode_step_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                       beta: torch.Tensor, state: torch.Tensor, *, options: int = 0, o: Optional[torch.Tensor] = None,
+                       dtype_o: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
+    """kda_decode_step_ex (include/kda.h): kda_decode_step with KDA_OPT_* options."""
+    return _decode("kda_decode_step_ex", q, k, v, log_alpha, beta, state, o, dtype_o, stream, options)
+
+
+def _decode(entry, q, k, v, log_alpha, beta, state, o, dtype_o, stream, options=0):
     lib = load_library()
     B, H, dk = q.shape
     dv = v.shape[2]
-    gate_shape = (B, H) if entry == "kda_gdn_decode_step" else (B, H, dk)
+    scalar_gate = entry == "kda_gdn_decode_step" or bool(options & KDA_OPT_SCALAR_GATE)
+    gate_shape = (B, H) if scalar_gate else (B, H, dk)
     if tuple(log_alpha.shape) != gate_shape:
         raise ValueError(f"log_alpha must be {list(gate_shape)}")
     if state.dtype != torch.float32 or state.shape != (B, H, dk, dv):
@@ -277,9 +306,10 @@ def _decode(entry, q, k, v, log_alpha, beta, state, o, dtype_o, stream):
         o = torch.empty((B, H, dv), dtype=dtype_o, device=q.device)
     _check_cuda(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, state=state, o=o), q.device)
     with torch.cuda.device(q.device):
+        extra = (int(options),) if entry == "kda_decode_step_ex" else ()
         st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state), B, H, dk, dv,
                                  _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"), _dtype_code(o, "o"),
-                                 _ptr(o), _stream_handle(stream))
+                                 _ptr(o), *extra, _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, entry)
     return o

@@ -189,6 +189,40 @@ KDA_API kda_status kda_gdn_decode_step(const void* q, const void* k, const void*
                            kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
                            void* o, void* stream);
 
+/* Options of kda_chunk_fwd_ex / kda_decode_step_ex (bitwise OR). */
+#define KDA_OPT_SCALAR_GATE 0x1u  /* log_alpha is [T_total, H] (resp. [B, H]): Gated DeltaNet, as
+                                     kda_gdn_chunk_fwd / kda_gdn_decode_step */
+#define KDA_OPT_L2NORM_QK 0x2u    /* q and k are raw: each (token, head) vector is divided by its
+                                     Euclidean length inside the kernels (in fp32, from the dtype_qkv
+                                     values; an all-zero vector stays zero) */
+#define KDA_OPT_BETA_LOGITS 0x4u  /* beta holds logits x: the kernels use beta = 1 / (1 + e^{-x}) */
+
+/*
+ * kda_chunk_fwd / kda_decode_step with the steps that come right before the operator in a KDA layer
+ * fused into its kernels.  Passage: "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)",
+ * section "Kimi Linear 모델 구성": queries and keys are L2-normalised (eigenvalue stability) before
+ * the KDA update, and the write strength beta lies in (0, 1).  The projections, short convolutions
+ * and the decay-gate function that produce q, k, beta and log_alpha need weights and are the
+ * caller's.
+ *   options     KDA_OPT_* bits; 0 gives exactly kda_chunk_fwd (resp. kda_decode_step).  Unknown bits
+ *               return KDA_ERR_INVALID_ARG.
+ * Every other argument, status and behaviour as kda_chunk_fwd (resp. kda_decode_step); with
+ * KDA_OPT_SCALAR_GATE log_alpha is laid out and aligned as for kda_gdn_chunk_fwd.
+ */
+KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                         const void* log_alpha, const void* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
+                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
+                         void* o, float* final_state,
+                         void* workspace, size_t workspace_bytes, uint32_t options, void* stream);
+
+KDA_API kda_status kda_decode_step_ex(const void* q, const void* k, const void* v,
+                           const void* log_alpha, const void* beta, float* state,
+                           int B, int H, int dk, int dv,
+                           kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
+                           void* o, uint32_t options, void* stream);
+
 /*
  * Waits for `stream`, then reads and clears the sticky device flags (KDA_DEVFLAG_*) of the current
  * device into *flags (may be NULL).  Returns KDA_OK if no flag was set, KDA_ERR_TIMEOUT if the

@@ -54,15 +54,34 @@ def max_threads() -> int:
     return int(_load().kda_oracle_max_threads())
 
 
+def l2_normalise(x):
+    """Each vector along the last axis divided by its Euclidean length (fp64); an all-zero vector stays
+    zero.  "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "Kimi Linear 모델 구성":
+    queries and keys are L2-normalised before the KDA update."""
+    x = _f64(x)
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return np.divide(x, n, out=np.zeros_like(x), where=n > 0)
+
+
+def sigmoid(x):
+    """The logistic function 1 / (1 + e^{-x}) (fp64): beta from its logit, in (0, 1)."""
+    return 1.0 / (1.0 + np.exp(-_f64(x)))
+
+
 def forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, rule=RULE_DELTA,
-            nthreads=0):
+            nthreads=0, l2norm_qk=False, beta_logits=False):
     """Sequential fp64 recurrence over a packed batch.
 
     Shapes: q, k, log_alpha [T, H, dk]; v [T, H, dv]; beta [T, H]; initial_state [N, H, dk, dv]
     or None (zeros); cu_seqlens [N+1] token offsets or None (one sequence of length T).
+    l2norm_qk: q and k are raw and are L2-normalised first; beta_logits: beta holds logits.
     Returns (o [T, H, dv], final_state [N, H, dk, dv]) as float64 numpy arrays.
     """
     q, k, v, la, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    if l2norm_qk:
+        q, k = l2_normalise(q), l2_normalise(k)
+    if beta_logits:
+        b = sigmoid(b)
     T, H, dk = q.shape
     dv = v.shape[2]
     if cu_seqlens is None:
@@ -88,10 +107,15 @@ def forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, rule=
     return o, sf
 
 
-def decode_step(q, k, v, log_alpha, beta, state, nthreads=0):
+def decode_step(q, k, v, log_alpha, beta, state, nthreads=0, l2norm_qk=False, beta_logits=False):
     """One recurrent step per (batch, head). q, k, log_alpha [B, H, dk]; v [B, H, dv]; beta [B, H];
-    state [B, H, dk, dv].  Returns (o [B, H, dv], new_state) as float64 numpy arrays."""
+    state [B, H, dk, dv].  l2norm_qk / beta_logits as in ``forward``.
+    Returns (o [B, H, dv], new_state) as float64 numpy arrays."""
     q, k, v, la, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    if l2norm_qk:
+        q, k = l2_normalise(q), l2_normalise(k)
+    if beta_logits:
+        b = sigmoid(b)
     S = _f64(state).copy()
     B, H, dk = q.shape
     dv = v.shape[2]
@@ -104,7 +128,7 @@ def decode_step(q, k, v, log_alpha, beta, state, nthreads=0):
     return o, S
 
 
-def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, nthreads=0):
+def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, nthreads=0, **prologue):
     """Gated DeltaNet over a packed batch: log_alpha [T, H] is one decay rate per token and head.
 
     "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "선형 어텐션에서 Gated
@@ -116,12 +140,12 @@ def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, n
     T, H, dk = _f64(q).shape
     assert la.shape == (T, H)
     return forward(q, k, v, np.repeat(la[:, :, None], dk, axis=2), beta, initial_state, cu_seqlens,
-                   nthreads=nthreads)
+                   nthreads=nthreads, **prologue)
 
 
-def gdn_decode_step(q, k, v, log_alpha, beta, state, nthreads=0):
+def gdn_decode_step(q, k, v, log_alpha, beta, state, nthreads=0, **prologue):
     """One Gated DeltaNet step: log_alpha [B, H], repeated over the key channels as in gdn_forward."""
     la = _f64(log_alpha)
     B, H, dk = _f64(q).shape
     assert la.shape == (B, H)
-    return decode_step(q, k, v, np.repeat(la[:, :, None], dk, axis=2), beta, state, nthreads=nthreads)
+    return decode_step(q, k, v, np.repeat(la[:, :, None], dk, axis=2), beta, state, nthreads=nthreads, **prologue)

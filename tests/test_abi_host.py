@@ -136,3 +136,16 @@ def test_static_scratch_rejects_oversize_before_any_cuda_call(lib):
     st = lib.kda_chunk_fwd_static_scratch(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 65536, 1, 4, 128, 128, 64,
                                           kda.KDA_BF16, kda.KDA_FP32, kda.KDA_FP32, FAKE, None, None)
     assert st == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_ex_entry_points_reject_unknown_options_on_host(lib):
+    st = lib.kda_chunk_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 128, 1, 2, 128, 128, 64, kda.KDA_BF16,
+                              kda.KDA_FP32, kda.KDA_FP32, FAKE, None, None, 0, 0x80, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    st = lib.kda_decode_step_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 128, kda.KDA_BF16, kda.KDA_FP32,
+                                kda.KDA_FP32, FAKE, 0x10, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    # the scalar-gate option relaxes log_alpha's alignment to its element size, as kda_gdn_chunk_fwd
+    st = lib.kda_chunk_fwd_ex(FAKE, FAKE, FAKE, FAKE + 2, FAKE, None, None, 128, 1, 2, 128, 128, 64, kda.KDA_BF16,
+                              kda.KDA_FP32, kda.KDA_FP32, FAKE, None, None, 0, kda.KDA_OPT_SCALAR_GATE, None)
+    assert st == kda.KDA_ERR_INVALID_ARG

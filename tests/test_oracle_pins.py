@@ -290,3 +290,61 @@ def test_invalid_arguments_are_rejected():
         oracle.forward(q, k, v, la, beta, None, np.array([0, 3, 2, 4]))
     with pytest.raises(ValueError):
         oracle.forward(q, k, v, la, beta, None, np.array([0, 5]))
+
+
+# ---------------------------------------------------------------- the fused prologue's definitions
+
+def test_l2norm_option_is_invariant_to_positive_row_scales_and_fixes_unit_rows():
+    """l2norm_qk=True: rescaling each (token, head) vector of q and k by a positive factor changes
+    nothing (a normalisation over any other axis would change), and rows that already have unit length
+    (Pythagorean-triple rows such as (3/5, 4/5)) give what they give with the option off; an all-zero
+    query row gives a zero output row."""
+    rng = np.random.default_rng(21)
+    T, H, dk, dv = 17, 2, 6, 3
+    q, k, v, la, beta, s0 = _rand_inputs(rng, T, H, dk, dv)
+    k = rng.standard_normal((T, H, dk))
+    a = np.exp(rng.uniform(-2, 2, (T, H, 1)))
+    b = np.exp(rng.uniform(-2, 2, (T, H, 1)))
+    o1, s1 = oracle.forward(q, k, v, la, beta, s0, l2norm_qk=True)
+    o2, s2 = oracle.forward(q * a, k * b, v, la, beta, s0, l2norm_qk=True)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(s2, s1, rtol=1e-12, atol=1e-13)
+    # unit rows: (3/5, 4/5) and (5/13, 12/13) placed in random channel pairs
+    qu, ku = np.zeros((T, H, dk)), np.zeros((T, H, dk))
+    for t in range(T):
+        for h in range(H):
+            i, j = rng.choice(dk, 2, replace=False)
+            qu[t, h, i], qu[t, h, j] = 0.6, 0.8
+            i, j = rng.choice(dk, 2, replace=False)
+            ku[t, h, i], ku[t, h, j] = 5 / 13, 12 / 13
+    o3, s3 = oracle.forward(qu, ku, v, la, beta, s0, l2norm_qk=True)
+    o4, s4 = oracle.forward(qu, ku, v, la, beta, s0)
+    np.testing.assert_allclose(o3, o4, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(s3, s4, rtol=1e-14, atol=1e-15)
+    q0 = q.copy()
+    q0[5, 1] = 0.0
+    o5, _ = oracle.forward(q0, k, v, la, beta, s0, l2norm_qk=True)
+    assert np.all(o5[5, 1] == 0.0)
+
+
+def test_beta_logits_option_is_the_logistic_function():
+    """beta_logits=True: logit 0 is beta = 1/2 exactly, and logits log(b / (1 - b)) reproduce the run
+    with beta = b (the inverse of the logistic function)."""
+    rng = np.random.default_rng(22)
+    T, H, dk, dv = 15, 2, 5, 4
+    q, k, v, la, beta, s0 = _rand_inputs(rng, T, H, dk, dv)
+    o1, s1 = oracle.forward(q, k, v, la, np.zeros((T, H)), s0, beta_logits=True)
+    o2, s2 = oracle.forward(q, k, v, la, np.full((T, H), 0.5), s0)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+    o3, s3 = oracle.forward(q, k, v, la, np.log(beta / (1 - beta)), s0, beta_logits=True)
+    o4, s4 = oracle.forward(q, k, v, la, beta, s0)
+    np.testing.assert_allclose(o3, o4, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(s3, s4, rtol=1e-12, atol=1e-13)
+    # decode: the same options on one step
+    od1, Sd1 = oracle.decode_step(q[:1], k[:1], v[:1], la[:1], np.zeros((1, H)), s0, beta_logits=True,
+                                  l2norm_qk=True)
+    od2, Sd2 = oracle.decode_step(oracle.l2_normalise(q[:1]), oracle.l2_normalise(k[:1]), v[:1], la[:1],
+                                  np.full((1, H), 0.5), s0)
+    np.testing.assert_array_equal(od1, od2)
+    np.testing.assert_array_equal(Sd1, Sd2)
