@@ -43,15 +43,27 @@ bool supported_dim(int d) { return d == 64 || d == 128; }
 
 }  // namespace
 
-constexpr uint32_t kKnownOptions = KDA_OPT_SCALAR_GATE | KDA_OPT_L2NORM_QK | KDA_OPT_BETA_LOGITS;
+constexpr uint32_t kKnownOptions =
+    KDA_OPT_SCALAR_GATE | KDA_OPT_L2NORM_QK | KDA_OPT_BETA_LOGITS | KDA_OPT_OUTPUT_NORM_GATE;
+
+// The epilogue's operands: present, aligned to their element size, eps finite and >= 0.
+bool epilogue_args_ok(uint32_t options, const void* out_gate, const float* norm_weight, float norm_eps,
+                      kda_dtype dtype_qkv, bool any_rows) {
+    if (!(options & KDA_OPT_OUTPUT_NORM_GATE)) return true;
+    if (!(norm_eps >= 0.f) || norm_eps > 3.0e38f) return false;
+    if (!any_rows) return true;
+    return out_gate && norm_weight && aligned_to(out_gate, dtype_size(dtype_qkv)) && aligned_to(norm_weight, 4);
+}
 
 // kda_chunk_fwd, kda_gdn_chunk_fwd and kda_chunk_fwd_ex (KDA_OPT_* options).
 kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                      const float* initial_state, const int32_t* cu_seqlens, int64_t T_total, int N, int H, int dk,
                      int dv, int chunk_size, kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
-                     float* final_state, void* workspace, size_t workspace_bytes, void* stream, uint32_t options) {
+                     float* final_state, void* workspace, size_t workspace_bytes, void* stream, uint32_t options,
+                     const void* out_gate = nullptr, const float* norm_weight = nullptr, float norm_eps = 0.f) {
     const bool scalar_gate = (options & KDA_OPT_SCALAR_GATE) != 0;
     if (options & ~kKnownOptions) return KDA_ERR_INVALID_ARG;
+    if (!epilogue_args_ok(options, out_gate, norm_weight, norm_eps, dtype_qkv, T_total > 0)) return KDA_ERR_INVALID_ARG;
     if (T_total < 0 || N <= 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk_size <= 0)
         return KDA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
@@ -83,26 +95,33 @@ kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* lo
     a.scalar_gate = scalar_gate;
     a.l2norm_qk = (options & KDA_OPT_L2NORM_QK) != 0;
     a.beta_logits = (options & KDA_OPT_BETA_LOGITS) != 0;
+    a.epilogue = (options & KDA_OPT_OUTPUT_NORM_GATE) != 0;
+    a.out_gate = out_gate; a.norm_weight = norm_weight; a.norm_eps = norm_eps;
     if (device_flags_ptr(&a.flags) != cudaSuccess) return KDA_ERR_CUDA;
 
     cudaError_t err;
+    bool epilogue_fused = false;
     if (!chunk_tc_supported(a)) {
         err = launch_chunk_simt(a);
     } else if (have_ws && need > 0) {
         err = launch_chunk_prep(a);
-        if (err == cudaSuccess) err = launch_chunk_scan(a);
+        if (err == cudaSuccess) err = launch_chunk_scan(a);  // the scan applies the epilogue itself
+        epilogue_fused = true;
     } else {
         err = launch_chunk_tc(a);
     }
+    if (err == cudaSuccess && a.epilogue && !epilogue_fused) err = launch_output_epilogue(a);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 // kda_decode_step, kda_gdn_decode_step and kda_decode_step_ex (KDA_OPT_* options).
 kda_status decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                        float* state, int B, int H, int dk, int dv, kda_dtype dtype_qkv, kda_dtype dtype_gate,
-                       kda_dtype dtype_o, void* o, void* stream, uint32_t options) {
+                       kda_dtype dtype_o, void* o, void* stream, uint32_t options, const void* out_gate = nullptr,
+                       const float* norm_weight = nullptr, float norm_eps = 0.f) {
     const bool scalar_gate = (options & KDA_OPT_SCALAR_GATE) != 0;
     if (options & ~kKnownOptions) return KDA_ERR_INVALID_ARG;
+    if (!epilogue_args_ok(options, out_gate, norm_weight, norm_eps, dtype_qkv, B > 0)) return KDA_ERR_INVALID_ARG;
     if (B < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype_qkv) || !valid_dtype(dtype_gate) || !valid_dtype(dtype_o))
         return KDA_ERR_INVALID_ARG;
@@ -124,6 +143,8 @@ kda_status decode_step(const void* q, const void* k, const void* v, const void* 
     a.scalar_gate = scalar_gate;
     a.l2norm_qk = (options & KDA_OPT_L2NORM_QK) != 0;
     a.beta_logits = (options & KDA_OPT_BETA_LOGITS) != 0;
+    a.epilogue = (options & KDA_OPT_OUTPUT_NORM_GATE) != 0;
+    a.out_gate = out_gate; a.norm_weight = norm_weight; a.norm_eps = norm_eps;
     return launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -176,17 +197,19 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
                             int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
                             kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
                             float* final_state, void* workspace, size_t workspace_bytes, uint32_t options,
-                            void* stream) {
+                            const void* out_gate, const float* norm_weight, float norm_eps, void* stream) {
     return kda::chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, T_total, N, H, dk, dv, chunk_size,
-                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, options);
+                          dtype_qkv, dtype_gate, dtype_o, o, final_state, workspace, workspace_bytes, stream, options,
+                          out_gate, norm_weight, norm_eps);
 }
 
 kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const void* log_alpha,
                               const void* beta, float* state, int B, int H, int dk, int dv,
                               kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
-                              uint32_t options, void* stream) {
+                              uint32_t options, const void* out_gate, const float* norm_weight, float norm_eps,
+                              void* stream) {
     return kda::decode_step(q, k, v, log_alpha, beta, state, B, H, dk, dv, dtype_qkv, dtype_gate, dtype_o, o,
-                            stream, options);
+                            stream, options, out_gate, norm_weight, norm_eps);
 }
 
 kda_status kda_get_device_status(void* stream, uint32_t* flags) {

@@ -57,7 +57,12 @@ constexpr uint32_t OFF_OST = 2 * STAGE_BYTES;   // o tile of one chunk, [64][64]
 constexpr uint32_t OFF_BARS = OFF_OST + 16384;  // full[2], empty[2], chain, sinit[2], odone[2]
 constexpr uint32_t OFF_SLOT = OFF_BARS + 9 * 8;
 constexpr uint32_t OFF_ABORT = OFF_SLOT + 4;
-constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
+// fused epilogue (EPI) only: per-token partial sums of squares
+constexpr uint32_t OFF_PEER = OFF_ABORT + 12;    // [2][64]: the other half's, written by it (by chunk parity)
+constexpr uint32_t OFF_QUAD = OFF_PEER + 512;    // [4][64]: this CTA's, per accumulator lane quadrant
+constexpr uint32_t OFF_INV = OFF_QUAD + 1024;    // [64]: 1 / rms of each token
+constexpr uint32_t OFF_PBAR = OFF_INV + 256;     // [2] mbarriers: the other half's sums arrived
+constexpr uint32_t SMEM_USED = OFF_PBAR + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 constexpr uint32_t TM_S = 0;    // state buffers at 0, 128, 256
@@ -97,11 +102,43 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// ---- the CTA pair of a head (a cluster of two, rank = value-column half) for the fused epilogue
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {  // same offset in CTA `rank`
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_peer_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t addr) {  // orders this thread's earlier peer stores
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// EPI: the fused output epilogue o <- o / rms(o) * w * sigmoid(gate) per (token, head), rms over all dv
+// value columns: launched as clusters of two (the head's two halves), which trade per-token partial
+// sums of squares through distributed shared memory.
+template <bool EPI>
 __global__ void __launch_bounds__(THREADS, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char* __restrict__ ws,
                   const float* initial_state,
                   const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H, void* __restrict__ o_ptr,
-                  int o_is_f32, float* final_state, unsigned int* flags) {
+                  int o_is_f32, float* final_state, unsigned int* flags, const void* __restrict__ out_gate,
+                  int gate_is_f32, const float* __restrict__ norm_weight, float norm_eps) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -133,12 +170,17 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
         mbar_init(sinit + 1, DATA_THREADS);
         mbar_init(odone, 1);
         mbar_init(odone + 1, 1);
+        if (EPI) {
+            mbar_init(reinterpret_cast<uint64_t*>(sm + OFF_PBAR), 64);
+            mbar_init(reinterpret_cast<uint64_t*>(sm + OFF_PBAR) + 1, 64);
+        }
         *abort = 0;
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(slot_tm, TM_COLS);
     tc_fence_before_sync();
     __syncthreads();
+    if (EPI) cluster_sync_all();  // both halves' barriers are initialised before either signals the other
     tc_fence_after_sync();
     const uint32_t tmem = *slot_tm;
 
@@ -159,10 +201,61 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             tmem_st32_x2<32>(tq + TM_S + 64 * g, v);
             tmem_st_wait();
         }
-        auto emit_o = [&](int c, const float (&x)[16]) {  // tokens 32 g + 16 hl .. +15 of O_c -> o
+        // epilogue operands of this lane: its weight, and the gates of the chunk it emits next
+        const float w_dv = EPI ? norm_weight[dv] : 1.f;
+        float pg[16];
+        auto fetch_gate = [&](int c) {  // tokens 32 g + 16 hl .. +15 of chunk c at value column dv
+            const int64_t c0 = t0 + static_cast<int64_t>(c) * C + 32 * g + 16 * hl;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int64_t idx = ((c0 + e) * H + h) * DV + dv;
+                pg[e] = c0 + e < t1 ? (gate_is_f32 ? static_cast<const float*>(out_gate)[idx]
+                                                   : __bfloat162float(static_cast<const __nv_bfloat16*>(out_gate)[idx]))
+                                    : 0.f;
+            }
+        };
+        auto emit_o = [&](int c, float (&x)[16]) {  // tokens 32 g + 16 hl .. +15 of O_c -> o
             const int64_t c0 = t0 + static_cast<int64_t>(c) * C;
             const int len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
             const int tb = 32 * g + 16 * hl;
+            if (EPI) {
+                // sum of x^2 over this CTA's 64 value columns per token: over the half-warp's 16 lanes by
+                // recursive halving (lane l & 15 ends with token tb + (l & 15)), then over the four warps
+                float v8[8], v4[4], v2[2];
+                const bool u8 = lane & 8, u4 = lane & 4, u2 = lane & 2, u1 = lane & 1;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float lo = x[i] * x[i], hi = x[i + 8] * x[i + 8];
+                    v8[i] = (u8 ? hi : lo) + __shfl_xor_sync(0xffffffffu, u8 ? lo : hi, 8);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) v4[i] = (u4 ? v8[i + 4] : v8[i]) + __shfl_xor_sync(0xffffffffu, u4 ? v8[i] : v8[i + 4], 4);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) v2[i] = (u2 ? v4[i + 2] : v4[i]) + __shfl_xor_sync(0xffffffffu, u2 ? v4[i] : v4[i + 2], 2);
+                const float v1 = (u1 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, u1 ? v2[0] : v2[1], 1);
+                float* quad = reinterpret_cast<float*>(sm + OFF_QUAD);
+                quad[(warp & 3) * 64 + tb + (lane & 15)] = v1;
+                group_sync(1, DATA_THREADS);
+                if (tid < 64) {  // token tid: this half's sum -> the other half; then both halves' sums
+                    const float mine = quad[tid] + quad[64 + tid] + quad[128 + tid] + quad[192 + tid];
+                    float* peer = reinterpret_cast<float*>(sm + OFF_PEER) + 64 * (c & 1);
+                    uint64_t* pbar = reinterpret_cast<uint64_t*>(sm + OFF_PBAR) + (c & 1);
+                    st_peer_f32(peer_addr(peer + tid, static_cast<uint32_t>(half ^ 1)), mine);
+                    mbar_arrive_peer(peer_addr(pbar, static_cast<uint32_t>(half ^ 1)));
+                    bool got = false;
+                    for (uint32_t i = 0; i < kWaitPolls && !got; ++i) {
+                        got = mbar_try_cluster(pbar, (c >> 1) & 1);
+                        if (!got && (i & 255u) == 255u && *abort) break;
+                    }
+                    if (!got) *abort = 1;
+                    const float ms = (mine + peer[tid]) * (1.f / static_cast<float>(DV));
+                    reinterpret_cast<float*>(sm + OFF_INV)[tid] = 1.f / sqrtf(ms + norm_eps);
+                }
+                group_sync(1, DATA_THREADS);
+                const float* inv = reinterpret_cast<const float*>(sm + OFF_INV);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) x[e] = x[e] * inv[tb + e] * w_dv * (1.f / (1.f + expf(-pg[e])));
+            }
             if (len == C) {  // whole chunk: rows into the o tile, then one TMA store
                 if (tid == 0) bulk_wait_read();  // the previous tile has left shared memory
                 group_sync(1, DATA_THREADS);
@@ -202,6 +295,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
         };
         bool ok = true;
         if (nc > 0) fetch(0);
+        if (EPI && nc > 0) fetch_gate(0);
         for (int c = 0; c < nc && ok; ++c) {
             // O_{c-2} out of output buffer c & 1 first, so chunk c's accumulators can be signalled before
             // O_{c-2} is written to memory
@@ -229,7 +323,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             tc_fence_before_sync();
             mbar_arrive(sinit + (c & 1));
             if (c + 1 < nc) fetch(c + 1);
-            if (c >= 2) emit_o(c - 2, ox);
+            if (c >= 2) {
+                emit_o(c - 2, ox);
+                if (EPI) fetch_gate(c - 1);
+            }
         }
         for (int c = nc - 2 < 0 ? 0 : nc - 2; c < nc && ok; ++c) {
             ok = wait_or_abort(odone + (c & 1), (c >> 1) & 1, abort);
@@ -238,6 +335,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             float ox[16];
             tmem_ld16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
             emit_o(c, ox);
+            if (EPI && c + 1 < nc) fetch_gate(c + 1);
         }
         if (ok && final_state) {  // after the last output MMA, the last state MMA is complete too
             const int i0 = 64 * g + 32 * hl;
@@ -319,6 +417,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
         tc_fence_after_sync();
         tmem_dealloc(tmem, TM_COLS);
     }
+    if (EPI) cluster_sync_all();  // neither half leaves while the other may still write into it
 }
 
 }  // namespace
@@ -330,14 +429,35 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
                         DV, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T_total), DVH, C,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    cudaError_t err =
-        cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (err != cudaSuccess) return err;
     const int64_t blocks = static_cast<int64_t>(a.N) * a.H * 2;
-    chunk_scan_kernel<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
-        mo, static_cast<const unsigned char*>(a.workspace), a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o,
-        a.dtype_o == KDA_FP32 ? 1 : 0, a.final_state, a.flags);
-    return cudaGetLastError();
+    const unsigned char* ws = static_cast<const unsigned char*>(a.workspace);
+    const int o32 = f32 ? 1 : 0, g32 = a.dtype_qkv == KDA_FP32 ? 1 : 0;
+    if (!a.epilogue) {
+        cudaError_t err = cudaFuncSetAttribute(chunk_scan_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        chunk_scan_kernel<false><<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
+            mo, ws, a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o, o32, a.final_state, a.flags, nullptr, 0,
+            nullptr, 0.f);
+        return cudaGetLastError();
+    }
+    cudaError_t err =
+        cudaFuncSetAttribute(chunk_scan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;  // the two value-column halves of one head
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chunk_scan_kernel<true>, mo, ws, a.initial_state, a.cu_seqlens, a.T_total, a.N,
+                              a.H, a.o, o32, a.final_state, a.flags, a.out_gate, g32, a.norm_weight, a.norm_eps);
 }
 
 }  // namespace kda

@@ -30,7 +30,8 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, 2)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                    const TG* __restrict__ log_alpha, const TG* __restrict__ beta,
                    float* __restrict__ state, TO* __restrict__ o, int scalar_gate, int l2norm_qk,
-                   int beta_logits) {
+                   int beta_logits, const TIn* __restrict__ out_gate, const float* __restrict__ norm_weight,
+                   float norm_eps) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int TPR = Sh::TPR, RG = Sh::RG, RPT = Sh::RPT;
 
@@ -39,6 +40,8 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     __shared__ __align__(16) float s_red_k[RG][DV];
     __shared__ __align__(16) float s_red_q[RG][DV];
     __shared__ float s_kq;
+    __shared__ float s_o[DV];  // o before the fused epilogue (out_gate != NULL)
+    __shared__ float s_inv;
 
     const int64_t u = blockIdx.x;  // (b, h) unit, row-major over [B, H]
     const int tid = threadIdx.x;
@@ -101,9 +104,23 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
         for (int g = 0; g < RG; ++g) { rk += s_red_k[g][j]; rq += s_red_q[g][j]; }
         const float d = b * (s_v[j] - rk);
         s_delta[j] = d;
-        o[u * DV + j] = from_f32<TO>(rq + d * s_kq);
+        if (out_gate) s_o[j] = rq + d * s_kq;
+        else o[u * DV + j] = from_f32<TO>(rq + d * s_kq);
     }
     __syncthreads();
+    if (out_gate) {  // fused epilogue: o / rms(o) * w * sigmoid(gate), rms over the dv values of the head
+        if (tid < 32) {
+            float ss = 0.f;
+            for (int j = tid; j < DV; j += 32) ss += s_o[j] * s_o[j];
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+            if (tid == 0) s_inv = 1.f / sqrtf(ss / static_cast<float>(DV) + norm_eps);
+        }
+        __syncthreads();
+        for (int j = tid; j < DV; j += Sh::THREADS)
+            o[u * DV + j] = from_f32<TO>(s_o[j] * s_inv * norm_weight[j] *
+                                         (1.f / (1.f + expf(-to_f32(out_gate[u * DV + j])))));
+    }
 
     const float4 d4 = reinterpret_cast<const float4*>(s_delta)[cg];
 #pragma unroll
@@ -121,7 +138,8 @@ cudaError_t launch_typed(const DecodeArgs& a) {
     decode_step_kernel<DK, DV, TIn, TG, TO><<<a.B * a.H, Sh::THREADS, 0, a.stream>>>(
         static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.v),
         static_cast<const TG*>(a.log_alpha), static_cast<const TG*>(a.beta), a.state,
-        static_cast<TO*>(a.o), a.scalar_gate ? 1 : 0, a.l2norm_qk ? 1 : 0, a.beta_logits ? 1 : 0);
+        static_cast<TO*>(a.o), a.scalar_gate ? 1 : 0, a.l2norm_qk ? 1 : 0, a.beta_logits ? 1 : 0,
+        a.epilogue ? static_cast<const TIn*>(a.out_gate) : nullptr, a.norm_weight, a.norm_eps);
     return cudaGetLastError();
 }
 

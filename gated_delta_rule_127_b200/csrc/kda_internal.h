@@ -28,6 +28,10 @@ struct ChunkArgs {
     bool scalar_gate;     // log_alpha is [T_total, H] (Gated DeltaNet), broadcast over dk
     bool l2norm_qk;       // q, k raw: divided by their L2 norm per (token, head) in the kernels
     bool beta_logits;     // beta holds logits: sigmoid applied in the kernels
+    bool epilogue;        // o <- o / rms(o) * norm_weight * sigmoid(out_gate) per (token, head)
+    const void* out_gate; // [T_total, H, dv], dtype_qkv
+    const float* norm_weight;  // [dv]
+    float norm_eps;
 };
 
 struct DecodeArgs {
@@ -45,6 +49,10 @@ struct DecodeArgs {
     bool scalar_gate;  // log_alpha is [B, H] (Gated DeltaNet), broadcast over dk
     bool l2norm_qk;    // q, k raw: divided by their L2 norm per (b, h) in the kernel
     bool beta_logits;  // beta holds logits: sigmoid applied in the kernel
+    bool epilogue;     // o <- o / rms(o) * norm_weight * sigmoid(out_gate) per (b, h)
+    const void* out_gate;  // [B, H, dv], dtype_qkv
+    const float* norm_weight;  // [dv]
+    float norm_eps;
 };
 
 // Each launcher returns cudaSuccess or the launch error.
@@ -58,5 +66,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a);
 size_t chunk_wy_workspace_size(int64_t T_total, int N, int H, int dk, int dv);
 cudaError_t launch_chunk_prep(const ChunkArgs& a);
 cudaError_t launch_chunk_scan(const ChunkArgs& a);
+// The output epilogue as its own pass over o, for the prefill paths that do not fuse it (the scan
+// does): o <- o / rms(o) * norm_weight * sigmoid(out_gate), one warp per (token, head).
+cudaError_t launch_output_epilogue(const ChunkArgs& a);
 
 }  // namespace kda

@@ -19,7 +19,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "kda.h")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_DEVICE_CHECK = range(6)
 KDA_BF16, KDA_FP32 = 0, 1
 KDA_DEVFLAG_CU_SEQLENS, KDA_DEVFLAG_DECAY_RANGE, KDA_DEVFLAG_TIMEOUT = 0x1, 0x2, 0x4
-KDA_OPT_SCALAR_GATE, KDA_OPT_L2NORM_QK, KDA_OPT_BETA_LOGITS = 0x1, 0x2, 0x4
+KDA_OPT_SCALAR_GATE, KDA_OPT_L2NORM_QK, KDA_OPT_BETA_LOGITS, KDA_OPT_OUTPUT_NORM_GATE = 0x1, 0x2, 0x4, 0x8
 
 _lib = None
 
@@ -53,9 +53,9 @@ def load_library() -> ctypes.CDLL:
     lib.kda_gdn_chunk_fwd.restype = i32
     lib.kda_gdn_decode_step.argtypes = lib.kda_decode_step.argtypes
     lib.kda_gdn_decode_step.restype = i32
-    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-1] + [ctypes.c_uint32, vp]
+    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes[:-1] + [ctypes.c_uint32, vp, vp, ctypes.c_float, vp]
     lib.kda_chunk_fwd_ex.restype = i32
-    lib.kda_decode_step_ex.argtypes = lib.kda_decode_step.argtypes[:-1] + [ctypes.c_uint32, vp]
+    lib.kda_decode_step_ex.argtypes = lib.kda_decode_step.argtypes[:-1] + [ctypes.c_uint32, vp, vp, ctypes.c_float, vp]
     lib.kda_decode_step_ex.restype = i32
     lib.kda_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.kda_get_device_status.restype = i32
@@ -156,16 +156,19 @@ def kda_chunk_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alph
                      chunk_size: int = 64, o: Optional[torch.Tensor] = None,
                      final_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
                      dtype_o: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
-                     use_workspace: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                     use_workspace: bool = True, out_gate: Optional[torch.Tensor] = None,
+                     norm_weight: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
+                     stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """kda_chunk_fwd_ex (include/kda.h): kda_chunk_fwd with KDA_OPT_* options (scalar gate, fused L2
-    normalisation of q and k, beta given as logits)."""
+    normalisation of q and k, beta given as logits, output RMSNorm + gate with out_gate [T, H, dv] in
+    q's dtype, norm_weight [dv] fp32 and norm_eps)."""
     return _chunk_fwd("kda_chunk_fwd_ex", q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs,
                       chunk_size, o, final_state, output_final_state, dtype_o, workspace, use_workspace, stream,
-                      options)
+                      options, (out_gate, norm_weight, norm_eps))
 
 
 def _chunk_fwd(entry, q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs, chunk_size, o, final_state,
-               output_final_state, dtype_o, workspace, use_workspace, stream, options=0):
+               output_final_state, dtype_o, workspace, use_workspace, stream, options=0, epi=(None, None, 0.0)):
     lib = load_library()
     scalar_gate = entry == "kda_gdn_chunk_fwd" or bool(options & KDA_OPT_SCALAR_GATE)
     gate_shape = q.shape[:2] if scalar_gate else q.shape
@@ -197,8 +200,11 @@ def _chunk_fwd(entry, q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_s
         raise ValueError("initial_state must be fp32 [N, H, dk, dv]")
     if final_state is not None and (final_state.dtype != torch.float32 or final_state.shape != (N, H, dk, dv)):
         raise ValueError("final_state must be fp32 [N, H, dk, dv]")
+    out_gate, norm_weight, norm_eps = epi
+    _check_epilogue(options, out_gate, norm_weight, (T, H, dv), q.dtype)
     _check_cuda(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, initial_state=initial_state,
-                     cu_seqlens=cu_seqlens, o=o, final_state=final_state, workspace=workspace), device)
+                     cu_seqlens=cu_seqlens, o=o, final_state=final_state, workspace=workspace, out_gate=out_gate,
+                     norm_weight=norm_weight), device)
     need = int(lib.kda_chunk_fwd_workspace_size(T, N, H, dk, dv, chunk_size))
     if not use_workspace:
         workspace = None
@@ -206,7 +212,7 @@ def _chunk_fwd(entry, q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_s
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(device):
-        extra = (int(options),) if entry == "kda_chunk_fwd_ex" else ()
+        extra = (int(options), _ptr(out_gate), _ptr(norm_weight), float(norm_eps)) if entry == "kda_chunk_fwd_ex" else ()
         st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
                                  _ptr(cu_seqlens), T, N, H, dk, dv, chunk_size,
                                  _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"), _dtype_code(o, "o"),
@@ -285,12 +291,25 @@ def kda_gdn_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a
 
 def kda_decode_step_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
                        beta: torch.Tensor, state: torch.Tensor, *, options: int = 0, o: Optional[torch.Tensor] = None,
-                       dtype_o: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
-    """kda_decode_step_ex (include/kda.h): kda_decode_step with KDA_OPT_* options."""
-    return _decode("kda_decode_step_ex", q, k, v, log_alpha, beta, state, o, dtype_o, stream, options)
+                       dtype_o: Optional[torch.dtype] = None, out_gate: Optional[torch.Tensor] = None,
+                       norm_weight: Optional[torch.Tensor] = None, norm_eps: float = 1e-6, stream=None) -> torch.Tensor:
+    """kda_decode_step_ex (include/kda.h): kda_decode_step with KDA_OPT_* options (out_gate [B, H, dv])."""
+    return _decode("kda_decode_step_ex", q, k, v, log_alpha, beta, state, o, dtype_o, stream, options,
+                   (out_gate, norm_weight, norm_eps))
 
 
-def _decode(entry, q, k, v, log_alpha, beta, state, o, dtype_o, stream, options=0):
+def _check_epilogue(options, out_gate, norm_weight, gate_shape, dtype):
+    if not options & KDA_OPT_OUTPUT_NORM_GATE:
+        return
+    if out_gate is None or norm_weight is None:
+        raise ValueError("KDA_OPT_OUTPUT_NORM_GATE needs out_gate and norm_weight")
+    if tuple(out_gate.shape) != tuple(gate_shape) or out_gate.dtype != dtype:
+        raise ValueError(f"out_gate must be {list(gate_shape)} in {dtype}")
+    if norm_weight.dtype != torch.float32 or tuple(norm_weight.shape) != (gate_shape[-1],):
+        raise ValueError("norm_weight must be fp32 [dv]")
+
+
+def _decode(entry, q, k, v, log_alpha, beta, state, o, dtype_o, stream, options=0, epi=(None, None, 0.0)):
     lib = load_library()
     B, H, dk = q.shape
     dv = v.shape[2]
@@ -304,9 +323,12 @@ def _decode(entry, q, k, v, log_alpha, beta, state, o, dtype_o, stream, options=
         dtype_o = o.dtype if o is not None else q.dtype
     if o is None:
         o = torch.empty((B, H, dv), dtype=dtype_o, device=q.device)
-    _check_cuda(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, state=state, o=o), q.device)
+    out_gate, norm_weight, norm_eps = epi
+    _check_epilogue(options, out_gate, norm_weight, (B, H, dv), q.dtype)
+    _check_cuda(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, state=state, o=o, out_gate=out_gate,
+                     norm_weight=norm_weight), q.device)
     with torch.cuda.device(q.device):
-        extra = (int(options),) if entry == "kda_decode_step_ex" else ()
+        extra = (int(options), _ptr(out_gate), _ptr(norm_weight), float(norm_eps)) if entry == "kda_decode_step_ex" else ()
         st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state), B, H, dk, dv,
                                  _dtype_code(q, "q"), _dtype_code(log_alpha, "log_alpha"), _dtype_code(o, "o"),
                                  _ptr(o), *extra, _stream_handle(stream))

@@ -196,16 +196,28 @@ KDA_API kda_status kda_gdn_decode_step(const void* q, const void* k, const void*
                                      Euclidean length inside the kernels (in fp32, from the dtype_qkv
                                      values; an all-zero vector stays zero) */
 #define KDA_OPT_BETA_LOGITS 0x4u  /* beta holds logits x: the kernels use beta = 1 / (1 + e^{-x}) */
+#define KDA_OPT_OUTPUT_NORM_GATE 0x8u  /* output epilogue: each (token, head) row of o becomes
+                                          o / sqrt(mean_j o_j^2 + norm_eps) * norm_weight
+                                          * sigmoid(out_gate) before it is stored */
 
 /*
- * kda_chunk_fwd / kda_decode_step with the steps that come right before the operator in a KDA layer
- * fused into its kernels.  Passage: "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)",
- * section "Kimi Linear 모델 구성": queries and keys are L2-normalised (eigenvalue stability) before
- * the KDA update, and the write strength beta lies in (0, 1).  The projections, short convolutions
- * and the decay-gate function that produce q, k, beta and log_alpha need weights and are the
- * caller's.
+ * kda_chunk_fwd / kda_decode_step with the steps that come right before and right after the operator
+ * in a KDA layer fused into its kernels.  Passage: "Kimi Linear: 표현력과 효율을 높인 어텐션
+ * 아키텍처(2025)", section "Kimi Linear 모델 구성": queries and keys are L2-normalised (eigenvalue
+ * stability) before the KDA update, the write strength beta lies in (0, 1), and before the output
+ * projection every head's output goes through RMSNorm and a data-dependent output gate.  The
+ * projections, short convolutions, the decay-gate function and the output gate's low-rank
+ * projection need weights and are the caller's: the gate arrives as its pre-activation values.
  *   options     KDA_OPT_* bits; 0 gives exactly kda_chunk_fwd (resp. kda_decode_step).  Unknown bits
  *               return KDA_ERR_INVALID_ARG.
+ *   out_gate    [T_total, H, dv] (resp. [B, H, dv]) dtype_qkv, the output gate's pre-activations;
+ *   norm_weight [dv] fp32, the RMSNorm weight shared by the heads;
+ *   norm_eps    >= 0, finite: all three read only with KDA_OPT_OUTPUT_NORM_GATE (then out_gate and
+ *               norm_weight must be non-NULL when there are rows, aligned to their element size).
+ *               On the bf16 dk = dv = 128 path with a workspace the epilogue runs inside the scan
+ *               (the two CTAs of a head form a cluster and trade per-token sums of squares); on the
+ *               other prefill paths it is a separate pass over o after the kernel, which with a bf16 o
+ *               normalises the rounded values.  The decode step applies it in its kernel.
  * Every other argument, status and behaviour as kda_chunk_fwd (resp. kda_decode_step); with
  * KDA_OPT_SCALAR_GATE log_alpha is laid out and aligned as for kda_gdn_chunk_fwd.
  */
@@ -215,13 +227,15 @@ KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                          int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
                          kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
                          void* o, float* final_state,
-                         void* workspace, size_t workspace_bytes, uint32_t options, void* stream);
+                         void* workspace, size_t workspace_bytes, uint32_t options,
+                         const void* out_gate, const float* norm_weight, float norm_eps, void* stream);
 
 KDA_API kda_status kda_decode_step_ex(const void* q, const void* k, const void* v,
                            const void* log_alpha, const void* beta, float* state,
                            int B, int H, int dk, int dv,
                            kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o,
-                           void* o, uint32_t options, void* stream);
+                           void* o, uint32_t options, const void* out_gate, const float* norm_weight,
+                           float norm_eps, void* stream);
 
 /*
  * Waits for `stream`, then reads and clears the sticky device flags (KDA_DEVFLAG_*) of the current

@@ -68,13 +68,24 @@ def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-_f64(x)))
 
 
+def output_epilogue(o, gate, weight, eps):
+    """Per-head RMSNorm and output gate on o [..., dv] (fp64): o / sqrt(mean_j o_j^2 + eps) * weight *
+    sigmoid(gate).  "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "Kimi Linear 모델
+    구성": before the output projection each head's output goes through RMSNorm and a data-dependent
+    output gate (read here as the logistic function of the given pre-activations)."""
+    o = _f64(o)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + float(eps))
+    return o / rms * _f64(weight) * sigmoid(gate)
+
+
 def forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, rule=RULE_DELTA,
-            nthreads=0, l2norm_qk=False, beta_logits=False):
+            nthreads=0, l2norm_qk=False, beta_logits=False, epilogue=None):
     """Sequential fp64 recurrence over a packed batch.
 
     Shapes: q, k, log_alpha [T, H, dk]; v [T, H, dv]; beta [T, H]; initial_state [N, H, dk, dv]
     or None (zeros); cu_seqlens [N+1] token offsets or None (one sequence of length T).
-    l2norm_qk: q and k are raw and are L2-normalised first; beta_logits: beta holds logits.
+    l2norm_qk: q and k are raw and are L2-normalised first; beta_logits: beta holds logits;
+    epilogue: None or (gate [T, H, dv], weight [dv], eps), applied to o by ``output_epilogue``.
     Returns (o [T, H, dv], final_state [N, H, dk, dv]) as float64 numpy arrays.
     """
     q, k, v, la, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
@@ -104,10 +115,12 @@ def forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, rule=
                                     _ptr(o), _ptr(sf), int(rule), int(nthreads))
     if rc != 0:
         raise ValueError(f"kda_oracle_forward failed with code {rc}")
+    if epilogue is not None:
+        o = output_epilogue(o, *epilogue)
     return o, sf
 
 
-def decode_step(q, k, v, log_alpha, beta, state, nthreads=0, l2norm_qk=False, beta_logits=False):
+def decode_step(q, k, v, log_alpha, beta, state, nthreads=0, l2norm_qk=False, beta_logits=False, epilogue=None):
     """One recurrent step per (batch, head). q, k, log_alpha [B, H, dk]; v [B, H, dv]; beta [B, H];
     state [B, H, dk, dv].  l2norm_qk / beta_logits as in ``forward``.
     Returns (o [B, H, dv], new_state) as float64 numpy arrays."""
@@ -125,6 +138,8 @@ def decode_step(q, k, v, log_alpha, beta, state, nthreads=0, l2norm_qk=False, be
                                    _ptr(o), int(nthreads))
     if rc != 0:
         raise ValueError(f"kda_oracle_decode failed with code {rc}")
+    if epilogue is not None:
+        o = output_epilogue(o, *epilogue)
     return o, S
 
 

@@ -139,13 +139,20 @@ def test_static_scratch_rejects_oversize_before_any_cuda_call(lib):
 
 
 def test_ex_entry_points_reject_unknown_options_on_host(lib):
-    st = lib.kda_chunk_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 128, 1, 2, 128, 128, 64, kda.KDA_BF16,
-                              kda.KDA_FP32, kda.KDA_FP32, FAKE, None, None, 0, 0x80, None)
-    assert st == kda.KDA_ERR_INVALID_ARG
+    ex = lambda opts, la=FAKE, g=None, w=None, eps=0.0: lib.kda_chunk_fwd_ex(
+        FAKE, FAKE, FAKE, la, FAKE, None, None, 128, 1, 2, 128, 128, 64, kda.KDA_BF16, kda.KDA_FP32, kda.KDA_FP32,
+        FAKE, None, None, 0, opts, g, w, eps, None)
+    assert ex(0x80) == kda.KDA_ERR_INVALID_ARG
     st = lib.kda_decode_step_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 128, kda.KDA_BF16, kda.KDA_FP32,
-                                kda.KDA_FP32, FAKE, 0x10, None)
+                                kda.KDA_FP32, FAKE, 0x10, None, None, 0.0, None)
     assert st == kda.KDA_ERR_INVALID_ARG
     # the scalar-gate option relaxes log_alpha's alignment to its element size, as kda_gdn_chunk_fwd
-    st = lib.kda_chunk_fwd_ex(FAKE, FAKE, FAKE, FAKE + 2, FAKE, None, None, 128, 1, 2, 128, 128, 64, kda.KDA_BF16,
-                              kda.KDA_FP32, kda.KDA_FP32, FAKE, None, None, 0, kda.KDA_OPT_SCALAR_GATE, None)
-    assert st == kda.KDA_ERR_INVALID_ARG
+    assert ex(kda.KDA_OPT_SCALAR_GATE, la=FAKE + 2) == kda.KDA_ERR_INVALID_ARG
+    # the epilogue needs its gate and weight, aligned, and a finite eps >= 0
+    E = kda.KDA_OPT_OUTPUT_NORM_GATE
+    assert ex(E, g=None, w=FAKE) == kda.KDA_ERR_INVALID_ARG
+    assert ex(E, g=FAKE, w=None) == kda.KDA_ERR_INVALID_ARG
+    assert ex(E, g=FAKE + 1, w=FAKE) == kda.KDA_ERR_INVALID_ARG
+    assert ex(E, g=FAKE, w=FAKE + 2) == kda.KDA_ERR_INVALID_ARG
+    assert ex(E, g=FAKE, w=FAKE, eps=-1.0) == kda.KDA_ERR_INVALID_ARG
+    assert ex(E, g=FAKE, w=FAKE, eps=float("nan")) == kda.KDA_ERR_INVALID_ARG

@@ -348,3 +348,29 @@ def test_beta_logits_option_is_the_logistic_function():
                                   np.full((1, H), 0.5), s0)
     np.testing.assert_array_equal(od1, od2)
     np.testing.assert_array_equal(Sd1, Sd2)
+
+
+def test_output_epilogue_is_a_per_head_rms_norm_and_gate():
+    """epilogue=(gate, w, eps): with eps = 0 scaling v and S0 by c > 0 (which scales o by c) changes
+    nothing; gate 0 halves, so 2 o' / w has unit root-mean-square over the dv values of every (token,
+    head) row -- a norm over any other axis, a sum for the mean or a different activation fails."""
+    rng = np.random.default_rng(23)
+    T, H, dk, dv = 13, 3, 5, 6
+    q, k, v, la, beta, s0 = _rand_inputs(rng, T, H, dk, dv)
+    gate = rng.standard_normal((T, H, dv))
+    w = np.exp(rng.uniform(-1, 1, dv))
+    o1, _ = oracle.forward(q, k, v, la, beta, s0, epilogue=(gate, w, 0.0))
+    o2, _ = oracle.forward(q, k, 7.5 * v, la, beta, 7.5 * s0, epilogue=(gate, w, 0.0))
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    o3, _ = oracle.forward(q, k, v, la, beta, s0, epilogue=(np.zeros((T, H, dv)), w, 0.0))
+    np.testing.assert_allclose(np.sqrt(np.mean((2 * o3 / w) ** 2, axis=-1)), 1.0, rtol=1e-13)
+    # eps: rows scaled so that mean(o^2) = m get exactly sqrt(m / (m + eps)) of the eps = 0 result
+    o_raw, _ = oracle.forward(q, k, v, la, beta, s0)
+    m = np.mean(o_raw ** 2, axis=-1, keepdims=True)
+    o4, _ = oracle.forward(q, k, v, la, beta, s0, epilogue=(gate, w, 0.25))
+    np.testing.assert_allclose(o4, o1 * np.sqrt(m / (m + 0.25)), rtol=1e-12, atol=1e-14)
+    od, _ = oracle.decode_step(q[:1], k[:1], v[:1], la[:1], beta[:1], s0, epilogue=(gate[:1], w, 0.0))
+    od_raw, _ = oracle.decode_step(q[:1], k[:1], v[:1], la[:1], beta[:1], s0)
+    np.testing.assert_allclose(np.sqrt(np.mean((od / (w * oracle.sigmoid(gate[:1]))) ** 2, axis=-1)), 1.0,
+                               rtol=1e-13)
+    assert np.all(np.sign(od) == np.sign(od_raw))
