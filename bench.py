@@ -45,8 +45,8 @@ PREFILL_KERNELS_PER_CALL = 2
 PREFILL_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_chunk_prep.cu",
                           "gated_delta_rule_127_b200/csrc/kda_chunk_scan.cu",
                           "gated_delta_rule_127_b200/csrc/kda_wy.cuh", "gated_delta_rule_127_b200/csrc/kda_sm100.cuh",
-                          "gated_delta_rule_127_b200/csrc/kda_tma.h"]
-DECODE_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_decode.cu"]
+                          "gated_delta_rule_127_b200/csrc/kda_tma.h", "gated_delta_rule_127_b200/csrc/kda_common.cuh"]
+DECODE_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_decode.cu", "gated_delta_rule_127_b200/csrc/kda_common.cuh"]
 
 
 def parse_args(argv=None):
