@@ -728,7 +728,8 @@ cudaError_t launch_prep(const ChunkArgs& a) {
 
 size_t chunk_wy_workspace_size(int64_t T_total, int N, int H, int dk, int dv) {
     if (T_total <= 0 || N <= 0 || H <= 0 || dk != DK || dv != DV) return 0;
-    return static_cast<size_t>(wy::num_slots(T_total, N)) * static_cast<size_t>(H) * wy::REC_BYTES;
+    return static_cast<size_t>(wy::num_slots(T_total, N)) * static_cast<size_t>(H) * wy::REC_BYTES +
+           chunk_scan_state_bytes(N, H);  // then the scan's states at the intra-sequence cut
 }
 
 template <bool SG>

@@ -132,13 +132,19 @@ __device__ __forceinline__ void cluster_sync_all() {
 // EPI: the fused output epilogue o <- o / rms(o) * w * sigmoid(gate) per (token, head), rms over all dv
 // value columns: launched as clusters of two (the head's two halves), which trade per-token partial
 // sums of squares through distributed shared memory.
-template <bool EPI>
+// Intra-sequence split (nseg = 2): each sequence's chunks are cut at mid = nc / 2.  A state-only pass
+// (SONLY: the state products alone, no output) runs the first part from S_0 and leaves the state at
+// the cut in s_mid, and a copy of S_0 in s0_copy; the full pass then runs both parts at once, CTA
+// segment 0 from the copy of S_0 and segment 1 from s_mid, so the sequential chain of the full pass
+// is half as long.  With nseg = 1 the full pass runs all chunks from S_0.
+template <bool EPI, bool SONLY>
 __global__ void __launch_bounds__(THREADS, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char* __restrict__ ws,
                   const float* initial_state,
                   const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H, void* __restrict__ o_ptr,
                   int o_is_f32, float* final_state, unsigned int* flags, const void* __restrict__ out_gate,
-                  int gate_is_f32, const float* __restrict__ norm_weight, float norm_eps) {
+                  int gate_is_f32, const float* __restrict__ norm_weight, float norm_eps, int nseg,
+                  float* __restrict__ s_mid, float* __restrict__ s0_copy) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -153,16 +159,26 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int half = static_cast<int>(blockIdx.x & 1);  // value columns 64 half .. +63
-    const int h = static_cast<int>((blockIdx.x >> 1) % H);
-    const int n = static_cast<int>((blockIdx.x >> 1) / H);
+    const int seg = SONLY ? 0 : static_cast<int>((blockIdx.x >> 1) % nseg);
+    const int unit = static_cast<int>((blockIdx.x >> 1) / (SONLY ? 1 : nseg));
+    const int h = unit % H;
+    const int n = unit / H;
     int64_t t0, t1;
     if (!wy::seq_bounds(cu_seqlens, T_total, N, n, t0, t1)) {
-        if (tid == 0) raise_flag(flags, KDA_DEVFLAG_CU_SEQLENS);
+        if (tid == 0 && seg == 0 && !SONLY) raise_flag(flags, KDA_DEVFLAG_CU_SEQLENS);
         return;
     }
-    const int nc = static_cast<int>((t1 - t0 + C - 1) / C);
-    const int64_t slot0 = wy::slot_base(t0, n);
+    const int nc_all = static_cast<int>((t1 - t0 + C - 1) / C), mid = nc_all / 2;
+    const int cb = (SONLY || nseg == 1 || seg == 0) ? 0 : mid;              // this CTA's chunks [cb, ce)
+    const int ce = SONLY ? mid : (nseg == 1 || seg == 1) ? nc_all : mid;
+    const int nc = ce - cb;
+    const int64_t slot0 = wy::slot_base(t0, n) + cb;  // record slot of local chunk 0
+    const int64_t tb0 = t0 + static_cast<int64_t>(cb) * C;  // first token of local chunk 0
     const int64_t state_off = (static_cast<int64_t>(n) * H + h) * DK * DV;
+    // where this CTA's start state comes from and its end state goes
+    const float* s_start = nseg == 1 ? initial_state : seg == 1 ? s_mid : (initial_state ? s0_copy : nullptr);
+    if (SONLY) s_start = initial_state;
+    float* s_end = SONLY ? s_mid : (seg == nseg - 1 ? final_state : nullptr);
 
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
@@ -197,7 +213,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             float v[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-                v[e] = initial_state ? initial_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] : 0.f;
+                v[e] = s_start ? s_start[state_off + static_cast<int64_t>(i0 + e) * DV + dv] : 0.f;
+            if (SONLY && initial_state) {  // the full pass's segment 0 starts from this copy
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s0_copy[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = v[e];
+            }
             tmem_st32_x2<32>(tq + TM_S + 64 * g, v);
             tmem_st_wait();
         }
@@ -205,7 +225,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
         const float w_dv = EPI ? norm_weight[dv] : 1.f;
         float pg[16];
         auto fetch_gate = [&](int c) {  // tokens 32 g + 16 hl .. +15 of chunk c at value column dv
-            const int64_t c0 = t0 + static_cast<int64_t>(c) * C + 32 * g + 16 * hl;
+            const int64_t c0 = tb0 + static_cast<int64_t>(c) * C + 32 * g + 16 * hl;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int64_t idx = ((c0 + e) * H + h) * DV + dv;
@@ -215,7 +235,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             }
         };
         auto emit_o = [&](int c, float (&x)[16]) {  // tokens 32 g + 16 hl .. +15 of O_c -> o
-            const int64_t c0 = t0 + static_cast<int64_t>(c) * C;
+            const int64_t c0 = tb0 + static_cast<int64_t>(c) * C;
             const int len = static_cast<int>((t1 - c0) < C ? (t1 - c0) : C);
             const int tb = 32 * g + 16 * hl;
             if (EPI) {
@@ -290,6 +310,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             const float4* gU = rec + wy::REC_UO / 16 + (8 * g + 4 * hl) * 128;
 #pragma unroll
             for (int s = 0; s < 8; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
+            if (SONLY) return;
 #pragma unroll
             for (int s = 0; s < 4; ++s) pu[s] = __ldcs(gU + s * 128 + dv);
         };
@@ -300,11 +321,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             // O_{c-2} out of output buffer c & 1 first, so chunk c's accumulators can be signalled before
             // O_{c-2} is written to memory
             float ox[16];
-            if (c >= 2) {
+            if (c >= 2) {  // (SONLY: odone marks the state product of the chunk, which freed the buffer)
                 ok = wait_or_abort(odone + (c & 1), ((c - 2) >> 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after_sync();
-                tmem_ld16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
+                if (!SONLY) tmem_ld16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
             }
             {
                 float vb[32], vu[16];
@@ -317,13 +338,13 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                     vu[4 * s] = pu[s].x; vu[4 * s + 1] = pu[s].y; vu[4 * s + 2] = pu[s].z; vu[4 * s + 3] = pu[s].w;
                 }
                 tmem_st32_x2<32>(tq + TM_S + 128 * ((c + 1) % 3) + 64 * g, vb);
-                tmem_st16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, vu);
+                if (!SONLY) tmem_st16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, vu);
             }
             tmem_st_wait();
             tc_fence_before_sync();
             mbar_arrive(sinit + (c & 1));
             if (c + 1 < nc) fetch(c + 1);
-            if (c >= 2) {
+            if (c >= 2 && !SONLY) {
                 emit_o(c - 2, ox);
                 if (EPI) fetch_gate(c - 1);
             }
@@ -332,17 +353,18 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             ok = wait_or_abort(odone + (c & 1), (c >> 1) & 1, abort);
             if (!ok) break;
             tc_fence_after_sync();
+            if (SONLY) continue;
             float ox[16];
             tmem_ld16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
             emit_o(c, ox);
             if (EPI && c + 1 < nc) fetch_gate(c + 1);
         }
-        if (ok && final_state) {  // after the last output MMA, the last state MMA is complete too
+        if (ok && s_end) {  // after the last output MMA (SONLY: state MMA), the last state MMA is complete too
             const int i0 = 64 * g + 32 * hl;
             float x[32];
             tmem_ld32_x2<32>(tq + TM_S + 128 * (nc % 3) + 64 * g, x);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) final_state[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = x[e];
+            for (int e = 0; e < 32; ++e) s_end[state_off + static_cast<int64_t>(i0 + e) * DV + dv] = x[e];
         }
     } else if (warp == LOADER_WARP) {
         // ---------------- loader: chunk c's Mt and Qh tiles into stage c & 1
@@ -353,16 +375,19 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                 if (c >= 2 && !wait_or_abort(empty + s, ((c - 2) >> 1) & 1, abort)) break;
                 const unsigned char* rec = ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES;
                 unsigned char* stage = sm + (s ? OFF_STAGE1 : OFF_STAGE0);
-                mbar_arrive_expect_tx(full + s, STAGE_BYTES);
+                mbar_arrive_expect_tx(full + s, SONLY ? 65536 : STAGE_BYTES);  // SONLY: Mt alone
 #pragma unroll
                 for (int b = 0; b < 4; ++b) bulk_load(stage + 16384 * b, rec + wy::REC_M + 16384 * b, 16384, full + s);
+                if (!SONLY) {
 #pragma unroll
-                for (int b = 0; b < 2; ++b)
-                    bulk_load(stage + 65536 + 16384 * b, rec + wy::REC_Q + 16384 * b, 16384, full + s);
-                if (c + 3 < nc) {  // the record three chunks ahead into L2
+                    for (int b = 0; b < 2; ++b)
+                        bulk_load(stage + 65536 + 16384 * b, rec + wy::REC_Q + 16384 * b, 16384, full + s);
+                }
+                if (c + 3 < nc) {  // the record three chunks ahead into L2 (SONLY: Mt and B)
                     const unsigned char* r3 = ws + (static_cast<size_t>(slot0 + c + 3) * H + h) * wy::REC_BYTES;
                     for (uint32_t off = 0; off < wy::REC_BYTES; off += 16384)
-                        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r3 + off), "r"(16384) : "memory");
+                        if (!SONLY || off < wy::REC_Q || (off >= wy::REC_B && off < wy::REC_UO))
+                            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r3 + off), "r"(16384) : "memory");
                 }
                 issued = c + 1;
             }
@@ -395,9 +420,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                 for (int kk = 0; kk < DK / 8; ++kk)  // K-step: 32 bytes within a 128-byte K-block
                     mma_tf32_ts(d_s, a_s + 8 * kk, bm + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), id_s, 1);
                 mma_commit(chain);
+                if (!SONLY) {
 #pragma unroll
-                for (int kk = 0; kk < DK / 8; ++kk)
-                    mma_tf32_ts(d_o, a_s + 8 * kk, bq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_o, 1);
+                    for (int kk = 0; kk < DK / 8; ++kk)
+                        mma_tf32_ts(d_o, a_s + 8 * kk, bq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_o, 1);
+                }
                 mma_commit(empty + s);
                 mma_commit(odone + s);
                 committed = c + 1;
@@ -422,6 +449,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
 
 }  // namespace
 
+size_t chunk_scan_state_bytes(int N, int H) {  // s_mid and the copy of S_0, fp32 [N, H, dk, dv] each
+    return 2 * static_cast<size_t>(N) * static_cast<size_t>(H) * DK * DV * sizeof(float);
+}
+
 cudaError_t launch_chunk_scan(const ChunkArgs& a) {
     CUtensorMap mo;
     const bool f32 = a.dtype_o == KDA_FP32;
@@ -429,35 +460,55 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
                         DV, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T_total), DVH, C,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const int64_t blocks = static_cast<int64_t>(a.N) * a.H * 2;
     const unsigned char* ws = static_cast<const unsigned char*>(a.workspace);
+    float* s_mid = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) +
+                                            static_cast<size_t>(wy::num_slots(a.T_total, a.N)) * a.H * wy::REC_BYTES);
+    float* s0_copy = s_mid + static_cast<size_t>(a.N) * a.H * DK * DV;
     const int o32 = f32 ? 1 : 0, g32 = a.dtype_qkv == KDA_FP32 ? 1 : 0;
-    if (!a.epilogue) {
-        cudaError_t err = cudaFuncSetAttribute(chunk_scan_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               SMEM_BYTES);
+    // Intra-sequence split when the (sequence, head) units leave most SMs idle: two segments per
+    // sequence need 4 CTAs per unit in one wave.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int nseg = 4 * static_cast<int64_t>(a.N) * a.H <= sms ? 2 : 1;
+    const int64_t units = static_cast<int64_t>(a.N) * a.H;
+    cudaError_t err;
+    if (nseg == 2) {  // the state at each sequence's cut, and a copy of S_0 for the first segment
+        err = cudaFuncSetAttribute(chunk_scan_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        chunk_scan_kernel<false><<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, a.stream>>>(
+        chunk_scan_kernel<false, true><<<static_cast<unsigned>(units * 2), THREADS, SMEM_BYTES, a.stream>>>(
             mo, ws, a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o, o32, a.final_state, a.flags, nullptr, 0,
-            nullptr, 0.f);
+            nullptr, 0.f, 1, s_mid, s0_copy);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+    const unsigned blocks = static_cast<unsigned>(units * 2 * nseg);
+    if (!a.epilogue) {
+        err = cudaFuncSetAttribute(chunk_scan_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        chunk_scan_kernel<false, false><<<blocks, THREADS, SMEM_BYTES, a.stream>>>(
+            mo, ws, a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o, o32, a.final_state, a.flags, nullptr, 0,
+            nullptr, 0.f, nseg, s_mid, s0_copy);
         return cudaGetLastError();
     }
-    cudaError_t err =
-        cudaFuncSetAttribute(chunk_scan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    err = cudaFuncSetAttribute(chunk_scan_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.gridDim = dim3(blocks, 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = a.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;  // the two value-column halves of one head
+    attr[0].val.clusterDim.x = 2;  // the two value-column halves of one head (and segment)
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, chunk_scan_kernel<true>, mo, ws, a.initial_state, a.cu_seqlens, a.T_total, a.N,
-                              a.H, a.o, o32, a.final_state, a.flags, a.out_gate, g32, a.norm_weight, a.norm_eps);
+    return cudaLaunchKernelEx(&cfg, chunk_scan_kernel<true, false>, mo, ws, a.initial_state, a.cu_seqlens, a.T_total,
+                              a.N, a.H, a.o, o32, a.final_state, a.flags, a.out_gate, g32, a.norm_weight, a.norm_eps,
+                              nseg, s_mid, s0_copy);
 }
 
 }  // namespace kda

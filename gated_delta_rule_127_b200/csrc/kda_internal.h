@@ -64,6 +64,8 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a);
 bool chunk_tc_supported(const ChunkArgs& a);
 cudaError_t launch_chunk_tc(const ChunkArgs& a);
 size_t chunk_wy_workspace_size(int64_t T_total, int N, int H, int dk, int dv);
+// The scan's part of that workspace, after the records: two fp32 [N, H, dk, dv] state arrays.
+size_t chunk_scan_state_bytes(int N, int H);
 cudaError_t launch_chunk_prep(const ChunkArgs& a);
 cudaError_t launch_chunk_scan(const ChunkArgs& a);
 // The output epilogue as its own pass over o, for the prefill paths that do not fuse it (the scan

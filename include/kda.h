@@ -120,9 +120,10 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
  * device code is loaded there, whose address is looked up once per device on the first call made
  * with that device current.
  *   - Limit: calls whose kda_chunk_fwd_workspace_size(...) exceeds KDA_STATIC_SCRATCH_BYTES return
- *     KDA_ERR_UNSUPPORTED before any CUDA call.  32 MiB holds 170 chunk records, one per 64-token
- *     chunk slot and head (slots = T_total / 64 + N + 1); e.g. 2 sequences x 2048 tokens x 2 heads
- *     uses 134.  Calls that need no workspace (fp32 q/k/v, dk or dv = 64) have no limit.
+ *     KDA_ERR_UNSUPPORTED before any CUDA call.  The size is one 192 KB chunk record per 64-token
+ *     chunk slot and head (slots = T_total / 64 + N + 1) plus 128 KB per (sequence, head); e.g. 2
+ *     sequences x 2048 tokens x 2 heads need 25.6 MiB.  Calls that need no workspace (fp32 q/k/v, dk
+ *     or dv = 64) have no limit.
  *   - Nothing in the scratch has to start at zero: every part a call reads is written earlier in the
  *     same call.
  *   - Every call on a device shares the one array: two calls that can run at the same time (on

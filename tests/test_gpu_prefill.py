@@ -209,3 +209,62 @@ def test_varlen_n16_h32_sampled():
     L = inp.lengths
     units = [(int(np.argmin(L)), 0), (int(np.argmax(L)), 31), (5, 7), (15, 16)]
     _check_units(inp, units, o, sf, torch.bfloat16)
+
+
+# ---------------------------------------------------------------- the scan's intra-sequence split
+
+def _embed_heads(inp, H_big, seed):
+    """The same sequences with the heads of `inp` as heads 0.. of a call with H_big heads (the others
+    random): enough (sequence, head) units that the scan runs each sequence in one piece."""
+    big = gen.make_prefill(inp.lengths, H_big, inp.dk, inp.dv, init_state=True, seed=seed, device=DEV)
+    H = inp.H
+    for name in ("q", "k", "v", "log_alpha", "beta", "initial_state"):
+        t = getattr(big, name)
+        if name == "initial_state":
+            t[:, :H] = inp.initial_state
+        else:
+            t[:, :H] = getattr(inp, name)
+    return big
+
+
+@pytest.mark.parametrize("epilogue", [False, True])
+def test_intra_sequence_split_is_bit_identical(epilogue):
+    """Few (sequence, head) units: the scan cuts each sequence in two (a state-only pass to the cut,
+    then both halves at once).  The same heads inside a 40-head call run uncut; the state products are
+    the same MMAs in the same order, so o and the final state agree bit for bit."""
+    inp = gen.make_prefill([700, 64, 1, 300, 0, 129], 2, 128, 128, init_state=True, seed=23, device=DEV)
+    big = _embed_heads(inp, 40, 24)
+    kw = dict(dtype_o=torch.float32)
+    if epilogue:
+        g = torch.Generator(device="cpu").manual_seed(5)
+        gate_big = torch.randn((big.T_total, 40, 128), generator=g).to(torch.bfloat16).to(DEV)
+        w = torch.exp(torch.rand((128,), generator=g) - 0.5).to(DEV)
+        kw.update(options=kda.KDA_OPT_OUTPUT_NORM_GATE, norm_weight=w, norm_eps=1e-6)
+        o1, s1 = kda.kda_chunk_fwd_ex(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state,
+                                      inp.cu_seqlens, out_gate=gate_big[:, :2].contiguous(), **kw)
+        o2, s2 = kda.kda_chunk_fwd_ex(big.q, big.k, big.v, big.log_alpha, big.beta, big.initial_state,
+                                      big.cu_seqlens, out_gate=gate_big, **kw)
+    else:
+        o1, s1 = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, inp.cu_seqlens,
+                                   **kw)
+        o2, s2 = kda.kda_chunk_fwd(big.q, big.k, big.v, big.log_alpha, big.beta, big.initial_state, big.cu_seqlens,
+                                   **kw)
+    assert kda.kda_get_device_status() == (kda.KDA_OK, 0)
+    assert torch.equal(o1, o2[:, :2]) and torch.equal(s1, s2[:, :2])
+
+
+def test_uncut_scan_matches_oracle():
+    """39 (sequence, head) units: every sequence is scanned in one piece."""
+    inp = gen.make_prefill([300, 70, 129], 13, 128, 128, init_state=True, seed=25, device=DEV)
+    _check_full(inp, torch.bfloat16)
+
+
+def test_split_with_aliased_state():
+    """final_state aliasing initial_state: the cut's first segment starts from a copy of S_0 taken before
+    any segment writes the final state."""
+    inp = gen.make_prefill([1000, 333], 2, 128, 128, init_state=True, seed=26, device=DEV)
+    o_ref, s_ref = _run(inp)
+    state = inp.initial_state.clone()
+    o, sf = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, state, inp.cu_seqlens,
+                              final_state=state, dtype_o=torch.float32)
+    assert torch.equal(o, o_ref) and torch.equal(state, s_ref)
