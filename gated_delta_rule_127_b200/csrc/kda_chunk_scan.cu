@@ -465,11 +465,15 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
                                             static_cast<size_t>(wy::num_slots(a.T_total, a.N)) * a.H * wy::REC_BYTES);
     float* s0_copy = s_mid + static_cast<size_t>(a.N) * a.H * DK * DV;
     const int o32 = f32 ? 1 : 0, g32 = a.dtype_qkv == KDA_FP32 ? 1 : 0;
-    // Intra-sequence split when the (sequence, head) units leave most SMs idle: two segments per
-    // sequence need 4 CTAs per unit in one wave.
+    // Intra-sequence split when there are few (sequence, head) units: the scan is then bound by each
+    // sequence's chain of chunks, not by the record stream.  With more units the CTAs already pull
+    // the records at a large share of HBM bandwidth (32 units: ~3.8 TB/s), and doubling the CTAs plus
+    // the state-only pass's extra Mt/B reads makes the call slower (32 units: 2.51 -> 2.69 ms).
+    constexpr int64_t kSplitMaxUnits = 8;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int nseg = 4 * static_cast<int64_t>(a.N) * a.H <= sms ? 2 : 1;
+    const int64_t nunits = static_cast<int64_t>(a.N) * a.H;
+    const int nseg = (nunits <= kSplitMaxUnits && 4 * nunits <= sms) ? 2 : 1;
     const int64_t units = static_cast<int64_t>(a.N) * a.H;
     cudaError_t err;
     if (nseg == 2) {  // the state at each sequence's cut, and a copy of S_0 for the first segment
