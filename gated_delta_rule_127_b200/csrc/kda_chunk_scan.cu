@@ -69,13 +69,14 @@ constexpr uint32_t TM_S = 0;    // state buffers at 0, 128, 256
 constexpr uint32_t TM_O = 384;  // output buffers at 384, 448
 constexpr uint32_t TM_COLS = 512;
 
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, 1); }
-
-// Bounded wait that also gives up when another role has flagged an abort; a timeout flags one.
+// Bounded wait (polls and wall time) that also gives up when another role has flagged an abort; a
+// timeout flags one.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    WaitBudget budget;
     for (uint32_t i = 0; i < kWaitPolls; ++i) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_poll(bar, parity)) return true;
         if ((i & 255u) == 255u && *abort) return false;
+        if (budget.expired()) break;
     }
     *abort = 1;
     return false;
@@ -263,9 +264,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                     st_peer_f32(peer_addr(peer + tid, static_cast<uint32_t>(half ^ 1)), mine);
                     mbar_arrive_peer(peer_addr(pbar, static_cast<uint32_t>(half ^ 1)));
                     bool got = false;
+                    WaitBudget budget;
                     for (uint32_t i = 0; i < kWaitPolls && !got; ++i) {
                         got = mbar_try_cluster(pbar, (c >> 1) & 1);
-                        if (!got && (i & 255u) == 255u && *abort) break;
+                        if (!got && (((i & 255u) == 255u && *abort) || budget.expired())) break;
                     }
                     if (!got) *abort = 1;
                     const float ms = (mine + peer[tid]) * (1.f / static_cast<float>(DV));

@@ -20,19 +20,50 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-// Bounded wait on phase `parity`; false if it did not complete within max_iter polls.
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Every bounded wait gives up after this much wall time (far above any legitimate wait, which is
+// microseconds).
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;
+
+// Elapsed-time bound for a polling loop: expired() after kWaitBudgetNs from the first call.
+struct WaitBudget {
+    uint64_t t0 = 0;
+    uint32_t polls = 0;
+    __device__ __forceinline__ bool expired() {
+        if ((polls++ & 63u) != 0) return false;  // read the timer every 64 polls
+        const uint64_t now = global_ns();
+        if (polls == 1) { t0 = now; return false; }
+        return now - t0 > kWaitBudgetNs;
+    }
+};
+
+// One poll of phase `parity` (the thread may be suspended for a system-dependent time while the phase
+// is incomplete); true once the phase completed.
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait on phase `parity`; false if it did not complete within max_iter polls or
+// kWaitBudgetNs of wall time, whichever comes first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter) {
-    const uint32_t addr = smem_u32(bar);
+    WaitBudget budget;
     for (uint32_t i = 0; i < max_iter; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.b32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
+        if (mbar_poll(bar, parity)) return true;
+        if (budget.expired()) return false;
     }
     return false;
 }
