@@ -98,3 +98,55 @@ def test_unmodified_source_passes_every_pin(tmp_path):
 def test_mutation_is_caught(tmp_path, name, old, new):
     fwd = _forward_with(_build_mutant(tmp_path, old, new))
     assert _failing_pins(fwd), f"no pin caught: {name}"
+
+
+# ---------------------------------------------------------------- the Python-side definitions
+# (name, function of the oracle module to replace, plausible wrong version, pins expected to catch it)
+PY_MUTATIONS = [
+    ("L2 norm over the token axis", "l2_normalise",
+     lambda x: oracle_mod._f64(x) / np.sqrt(np.sum(oracle_mod._f64(x) ** 2, axis=0, keepdims=True))),
+    ("L2 norm divides by the squared norm", "l2_normalise",
+     lambda x: oracle_mod._f64(x) / np.sum(oracle_mod._f64(x) ** 2, axis=-1, keepdims=True)),
+    ("sigmoid of -x", "sigmoid", lambda x: 1.0 / (1.0 + np.exp(oracle_mod._f64(x)))),
+    ("tanh instead of the logistic function", "sigmoid", lambda x: 0.5 * (1.0 + np.tanh(oracle_mod._f64(x)))),
+    ("RMS from the sum of squares", "output_epilogue",
+     lambda o, g, w, eps: oracle_mod._f64(o) / np.sqrt(np.sum(oracle_mod._f64(o) ** 2, axis=-1, keepdims=True) + eps)
+     * oracle_mod._f64(w) * oracle_mod.sigmoid(g)),
+    ("RMS over the head axis", "output_epilogue",
+     lambda o, g, w, eps: oracle_mod._f64(o) / np.sqrt(np.mean(oracle_mod._f64(o) ** 2, axis=-2, keepdims=True) + eps)
+     * oracle_mod._f64(w) * oracle_mod.sigmoid(g)),
+    ("eps outside the square root", "output_epilogue",
+     lambda o, g, w, eps: oracle_mod._f64(o) / (np.sqrt(np.mean(oracle_mod._f64(o) ** 2, axis=-1, keepdims=True)) + eps)
+     * oracle_mod._f64(w) * oracle_mod.sigmoid(g)),
+]
+
+PY_PINS = [pins.test_l2norm_option_is_invariant_to_positive_row_scales_and_fixes_unit_rows,
+           pins.test_beta_logits_option_is_the_logistic_function,
+           pins.test_output_epilogue_is_a_per_head_rms_norm_and_gate]
+
+
+@pytest.mark.parametrize("name,func,bad", [m[:3] for m in PY_MUTATIONS], ids=[m[0] for m in PY_MUTATIONS])
+def test_python_side_mutation_is_caught(monkeypatch, name, func, bad):
+    for pin in PY_PINS:  # the unmodified definitions pass
+        pin()
+    monkeypatch.setattr(oracle_mod, func, bad)
+    caught = []
+    for pin in PY_PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught: {name}"
+
+
+def test_gdn_gate_taken_as_alpha_is_caught(monkeypatch):
+    """A GDN front end that forgets the gate is a log (passes alpha where log alpha belongs) fails the
+    textbook-recurrence pin."""
+    pins.test_gdn_entry_points_follow_the_textbook_recurrence()
+    real = oracle_mod.gdn_forward
+
+    def wrong(q, k, v, log_alpha, beta, *a, **kw):
+        return real(q, k, v, np.exp(oracle_mod._f64(log_alpha)), beta, *a, **kw)
+    monkeypatch.setattr(oracle, "gdn_forward", wrong)
+    with pytest.raises(AssertionError):
+        pins.test_gdn_entry_points_follow_the_textbook_recurrence()
