@@ -235,6 +235,19 @@ def oracle_sample_rate(inp, n_units: int, tokens: int):
     return len(args) * tokens / dt, threads, dt
 
 
+# The metric and workload description both arms report (the reference arm times the oracle on a
+# bounded sample of the same workload; its `cpu_baseline.sample` says which).
+METRIC = "KDA chunked-prefill tokens/s (decode-step state GB/s in 'decode')"
+
+
+def workload_config(world: int) -> dict:
+    return {"workload": f"{PREFILL}: B=1, H=32, T=32768, dk=dv=128, chunk 64, bf16 q/k/v, fp32 "
+                        f"log_alpha/beta, bf16 o; plus one {DECODE} step (256 x 32 fp32 128x128 "
+                        f"states) per step",
+            "l2": "no flush: every input is larger than L2 (prefill 1.6 GB, decode state 537 MB)",
+            "parallelism": f"independent replica per GPU x{world}"}
+
+
 # ------------------------------------------------------------------------------------ reference arm
 
 def run_reference(args):
@@ -258,11 +271,11 @@ def run_reference(args):
     value = tok_heads_per_s / w["H"]  # tokens/s of the H-head workload
     sample = f"{n_units} (head) units x first {tokens} tokens of {PREFILL} per step, fp64 sequential recurrence"
     line = {
-        "impl": "reference", "metric": "KDA chunked-prefill tokens/s (fp64 CPU oracle)", "value": value,
+        "impl": "reference", "metric": METRIC, "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * n_units * tokens / tok_heads_per_s, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{PREFILL} (B=1, H=32, T=32768, dk=dv=128, chunk 64)"},
+        "config": workload_config(args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -408,7 +421,7 @@ def run_ours(args):
                    "sample": f"{n_units} (head) units x all 32768 tokens of {PREFILL} ({secs:.1f} s wall, "
                              f"fp64 sequential recurrence, OpenMP over units)"}
         line = {
-            "metric": "KDA chunked-prefill tokens/s (decode-step state GB/s in 'decode')",
+            "metric": METRIC,
             "value": world * T * 1000.0 / prefill_max,
             "unit": "tokens/s",
             "n_gpus": world,
@@ -420,11 +433,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{PREFILL}: B=1, H=32, T=32768, dk=dv=128, chunk 64, bf16 q/k/v, fp32 "
-                                   f"log_alpha/beta, bf16 o; plus one {DECODE} step (256 x 32 fp32 128x128 "
-                                   f"states) per step",
-                       "l2": "no flush: every input is larger than L2 (prefill 1.6 GB, decode state 537 MB)",
-                       "parallelism": f"independent replica per GPU x{world}"},
+            "config": workload_config(world),
             "prefill_ms": prefill_max,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved_gbs / hbm_peak, "traffic": traffic,

@@ -10,10 +10,11 @@
 //   K+ = K e^{G - g_m},  Q+ = Q e^{G - g_m},  K- = K e^{g_m - G}         elementwise, fp32
 //   [A_raw; P] = [K+; Q+] (K-)^T                                         MMA 1 (A operand in TMEM)
 //   A = beta_r A_raw strictly lower, P lower with the diagonal
-//   T = (I + A)^{-1}: 16 x 16 diagonal blocks by forward substitution, then merged into 32 x 32 and
-//       64 x 64 inverses with [[T1, 0], [-T2 A21 T1, T2]]                                fp32
+//   T = (I + A)^{-1}: 16 x 16 diagonal blocks by forward substitution (fp32), then merged into
+//       32 x 32 and 64 x 64 inverses with [[T1, 0], [-T2 A21 T1, T2]] on warp-level tensor-core
+//       tiles (mma.sync tf32, fp32 accumulation)
 //   [W | U] = T [beta K e^G | beta V]                                    MMA 2
-//   P W,  Kt^T W,  B^T = U^T Kt,  Uo^T = U^T P^T                          MMAs 3-6
+//   B^T = U^T Kt,  Uo^T = U^T P^T (MMAs 5-6, first),  P W,  Kt^T W (MMAs 3-4)
 //   Mt = Diag(e^{g_C}) - Kt^T W,  Qh = Q e^G - P W
 // B and Uo are formed transposed so that the accumulator lane is the value column: they go from
 // registers straight to memory in contiguous runs.  Mt and Qh are staged in shared memory as the
@@ -25,10 +26,14 @@
 // accumulation (operands rounded to tf32 when written); B and Uo are stored in fp32.
 //
 // Persistent CTAs of 512 threads, one per SM, each taking (chunk slot, head) tasks in turn.  The next
-// task's input tiles are loaded into shared memory while the task's results are being stored.  Elementwise pass: thread t owns key
-// channel c = 32 (w % 4) + lane (its tensor-memory lane, w = warp) and rows 16 (w / 4) .. +15, so the
-// cumulative sum runs down a column in registers.  Row pass and accumulator read-outs: the warp's
-// lane quadrant gives the row, w / 4 the column quarter.
+// task's input tiles are loaded into shared memory while the task's results are being stored.
+// Elementwise pass: thread t owns key channel c = 32 (w % 4) + lane (its tensor-memory lane, w =
+// warp) and rows 16 (w / 4) .. +15, so the cumulative sum runs down a column in registers.  Row pass
+// and accumulator read-outs: the warp's lane quadrant gives the row, w / 4 the column quarter (M = 64
+// accumulators through the 16x32bx2 shape, lanes 16..31 taking a second column range).
+// Template options: TG the gate dtype; SG Gated DeltaNet's scalar gate (one rate per token and head,
+// read with beta, broadcast over the channels in the cumulative sum); PRO the fused L2 normalisation
+// of q and k (each use of a row scaled by 1 / its norm).
 #include <cuda_bf16.h>
 
 #include "kda_common.cuh"

@@ -23,8 +23,9 @@
 // 16..31 reach the same rows through the 16x32bx2 access shape at a column offset) and half w / 4 of
 // the accumulator columns, and holds the next chunk's share of B and Uo in registers while the
 // current chunk's MMAs run; warp 8 lane 0 brings each chunk's Mt and Qh operand tiles into a two-stage
-// shared-memory ring with bulk copies (and asks L2 for the B and Uo of the chunk after); warp 9
-// lane 0 issues the MMAs.
+// shared-memory ring with bulk copies (and asks L2 for the record three chunks ahead); warp 9
+// lane 0 issues the MMAs.  Further options: the fused output epilogue (EPI, a cluster of two per head)
+// and the intra-sequence split (SONLY state-only pass plus nseg = 2 segments), described at the kernel.
 // Tensor memory: three state buffers (S_n read while S_{n+1} accumulates and S_{n+2}'s B is written)
 // and two output buffers.
 #include <cuda_bf16.h>
@@ -312,9 +313,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             const float4* gU = rec + wy::REC_UO / 16 + (8 * g + 4 * hl) * 128;
 #pragma unroll
             for (int s = 0; s < 8; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
-            if (SONLY) return;
+            if (!SONLY) {  // the state-only pass has no output
 #pragma unroll
-            for (int s = 0; s < 4; ++s) pu[s] = __ldcs(gU + s * 128 + dv);
+                for (int s = 0; s < 4; ++s) pu[s] = __ldcs(gU + s * 128 + dv);
+            }
         };
         bool ok = true;
         if (nc > 0) fetch(0);

@@ -105,12 +105,6 @@ __device__ __forceinline__ void st_mn8(unsigned char* base, uint32_t off, int k_
     d[1] = make_float4(to_tf32(x[4]), to_tf32(x[5]), to_tf32(x[6]), to_tf32(x[7]));
 }
 
-// Four consecutive M/N elements (col multiple of 4) of one K-row of an MN-major tile, rounded to tf32.
-__device__ __forceinline__ void st_mn4(unsigned char* base, uint32_t off, int k_row, int col, int rows,
-                                       const float* x) {
-    *reinterpret_cast<float4*>(base + off + sw32b_off(k_row, col, rows)) =
-        make_float4(to_tf32(x[0]), to_tf32(x[1]), to_tf32(x[2]), to_tf32(x[3]));
-}
 // Four consecutive elements (col multiple of 4) of one row of a K-major tile, rounded to tf32.
 __device__ __forceinline__ void st_sw4(unsigned char* base, uint32_t off, int row, int col, int rows,
                                        float a, float b, float c, float d) {
