@@ -23,7 +23,8 @@
 // below e^80 while the chunk's log-decay stays within 80 of g_m at both ends ("일반 DPLR보다 줄어든
 // 연산량" on the same page notes that fine-grained decay makes intra-chunk division delicate);
 // outside that range the chunk sets KDA_DEVFLAG_DECAY_RANGE.  Every MMA runs kind::tf32 with fp32
-// accumulation (operands rounded to tf32 when written); B and Uo are stored in fp32.
+// accumulation (operands rounded to tf32 when written); B is stored in fp16 with a power-of-two
+// exponent per 32 rows and value column (fp16 keeps tf32's 10-bit mantissa), Uo in fp32.
 //
 // Persistent CTAs of 512 threads, one per SM, each taking (chunk slot, head) tasks in turn.  The next
 // task's input tiles are loaded into shared memory while the task's results are being stored.
@@ -35,6 +36,7 @@
 // read with beta, broadcast over the channels in the cumulative sum); PRO the fused L2 normalisation
 // of q and k (each use of a row scaled by 1 / its norm).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -608,10 +610,25 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record
             float x[32];
             tmem_ld32(tq + TM_BT + 32 * qr, x);
-            float4* gb = reinterpret_cast<float4*>(rec + wy::REC_B);
+            float m = 0.f;
 #pragma unroll
-            for (int s4 = 0; s4 < 8; ++s4)
-                gb[(8 * qr + s4) * 128 + c] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
+            for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(x[e]));
+            // B in fp16: the 32 rows' largest magnitude scaled into [2^14, 2^15) by a power of two
+            int ex = static_cast<int>((__float_as_uint(m) >> 23) & 0xffu) - 127 - 14;
+            ex = ex < -100 ? -100 : ex > 100 ? 100 : ex;
+            const float sc = __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);  // 2^-ex
+            uint4* gb = reinterpret_cast<uint4*>(rec + wy::REC_B);
+#pragma unroll
+            for (int s8 = 0; s8 < 4; ++s8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const __half2 hv = __floats2half2_rn(x[8 * s8 + 2 * p] * sc, x[8 * s8 + 2 * p + 1] * sc);
+                    w[p] = *reinterpret_cast<const uint32_t*>(&hv);
+                }
+                gb[(4 * qr + s8) * 128 + c] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            reinterpret_cast<signed char*>(rec + wy::REC_BEXP)[qr * 128 + c] = static_cast<signed char>(ex);
             float y[16];
             tmem_ld16(tq + TM_UT + 16 * qr, y);
             float4* gu = reinterpret_cast<float4*>(rec + wy::REC_UO);

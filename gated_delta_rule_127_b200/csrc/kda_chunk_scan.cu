@@ -29,6 +29,7 @@
 // Tensor memory: three state buffers (S_n read while S_{n+1} accumulates and S_{n+2}'s B is written)
 // and two output buffers.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -305,14 +306,17 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
         };
         // this lane's share of chunk c's B^T (rows i = 64 g + 32 hl .. +31) and Uo^T (tokens 32 g + 16 hl
         // .. +15), loaded one chunk ahead
-        float4 pb[8], pu[4];
+        uint4 pb[4];  // B rows i = 64 g + 32 hl .. +31 in fp16, scaled by 2^-pe
+        float4 pu[4];
+        int pe = 0;
         auto fetch = [&](int c) {
             const float4* rec =
                 reinterpret_cast<const float4*>(ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES);
-            const float4* gB = rec + wy::REC_B / 16 + (16 * g + 8 * hl) * 128;
+            const uint4* gB = reinterpret_cast<const uint4*>(rec + wy::REC_B / 16) + (8 * g + 4 * hl) * 128;
             const float4* gU = rec + wy::REC_UO / 16 + (8 * g + 4 * hl) * 128;
 #pragma unroll
-            for (int s = 0; s < 8; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
+            for (int s = 0; s < 4; ++s) pb[s] = __ldcs(gB + s * 128 + dv);
+            pe = reinterpret_cast<const signed char*>(rec + wy::REC_BEXP / 16)[(2 * g + hl) * 128 + dv];
             if (!SONLY) {  // the state-only pass has no output
 #pragma unroll
                 for (int s = 0; s < 4; ++s) pu[s] = __ldcs(gU + s * 128 + dv);
@@ -333,9 +337,16 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             }
             {
                 float vb[32], vu[16];
+                const float sc = __uint_as_float(static_cast<uint32_t>(127 + pe) << 23);  // 2^pe
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    vb[4 * s] = pb[s].x; vb[4 * s + 1] = pb[s].y; vb[4 * s + 2] = pb[s].z; vb[4 * s + 3] = pb[s].w;
+                for (int s = 0; s < 4; ++s) {
+                    const uint32_t w[4] = {pb[s].x, pb[s].y, pb[s].z, pb[s].w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
+                        vb[8 * s + 2 * p] = f.x * sc;
+                        vb[8 * s + 2 * p + 1] = f.y * sc;
+                    }
                 }
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
@@ -390,8 +401,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                 if (c + 3 < nc) {  // the record three chunks ahead into L2 (SONLY: Mt and B)
                     const unsigned char* r3 = ws + (static_cast<size_t>(slot0 + c + 3) * H + h) * wy::REC_BYTES;
                     for (uint32_t off = 0; off < wy::REC_BYTES; off += 16384)
-                        if (!SONLY || off < wy::REC_Q || (off >= wy::REC_B && off < wy::REC_UO))
-                            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r3 + off), "r"(16384) : "memory");
+                        if (!SONLY || off < wy::REC_Q || (off >= wy::REC_B && off < wy::REC_UO) || off >= wy::REC_BEXP)
+                            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r3 + off),
+                                         "r"(wy::REC_BYTES - off < 16384u ? wy::REC_BYTES - off : 16384u)
+                                         : "memory");
                 }
                 issued = c + 1;
             }

@@ -16,10 +16,15 @@
 //          sw128_off(i, j, 128).  Rounded to tf32.
 //   REC_Q  Qh as the scan's B operand (K = j, N = token t): four K-blocks of 64 rows x 128 bytes;
 //          element (t, j) at sw128_off(t, j, 64).  Rounded to tf32.
-//   REC_B  B transposed and interleaved by four: element (i, dv) at float index (i / 4) * 512 + dv * 4
-//          + i % 4, so thread dv reading float4 number (i / 4) * 128 + dv gets B[i..i+3][dv] and a
-//          warp's read, like the writer's store of four rows, is one contiguous 512-byte run.
-//   REC_UO Uo the same way: element (t, dv) at float index (t / 4) * 512 + dv * 4 + t % 4.
+//   REC_B  B transposed, in fp16 with a power-of-two scale per 32 rows and value column, interleaved
+//          by eight: element (i, dv) is B[i][dv] * 2^-e at half index (i / 8) * 1024 + dv * 8 + i % 8,
+//          so thread dv reading 16 bytes at uint4 number (i / 8) * 128 + dv gets rows i..i+7 and a
+//          warp's read, like the writer's store, is one contiguous 512-byte run.  fp16 keeps tf32's
+//          10-bit mantissa; e (signed byte at REC_BEXP + (i / 32) * 128 + dv) puts the group's
+//          largest magnitude in [2^14, 2^15), so no value of the group overflows or loses relative
+//          precision unless it is 2^-28 times smaller than the largest.
+//   REC_UO Uo in fp32, interleaved by four: element (t, dv) at float index (t / 4) * 512 + dv * 4 + t % 4
+//          (thread dv's float4 number (t / 4) * 128 + dv is Uo[t..t+3][dv]).
 // Chunk c of sequence n has slot  floor(cu[n] / 64) + n + c;  the record of (slot, head h) starts at
 // (slot * H + h) * REC_BYTES.  The slot map is one-to-one because floor(cu[n+1]/64) >= floor(cu[n]/64)
 // + ceil(L_n/64) - 1, and slots stay below T_total / 64 + N + 1.
@@ -36,8 +41,9 @@ constexpr int DV = 128;
 constexpr uint32_t REC_M = 0;
 constexpr uint32_t REC_Q = 65536;
 constexpr uint32_t REC_B = 98304;
-constexpr uint32_t REC_UO = 163840;
-constexpr uint32_t REC_BYTES = 196608;
+constexpr uint32_t REC_UO = 131072;
+constexpr uint32_t REC_BEXP = 163840;
+constexpr uint32_t REC_BYTES = 164352;
 
 __host__ __device__ constexpr int64_t num_slots(int64_t T_total, int N) { return T_total / C + N + 1; }
 

@@ -120,9 +120,9 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
  * device code is loaded there, whose address is looked up once per device on the first call made
  * with that device current.
  *   - Limit: calls whose kda_chunk_fwd_workspace_size(...) exceeds KDA_STATIC_SCRATCH_BYTES return
- *     KDA_ERR_UNSUPPORTED before any CUDA call.  The size is one 192 KB chunk record per 64-token
+ *     KDA_ERR_UNSUPPORTED before any CUDA call.  The size is one 160.5 KB chunk record per 64-token
  *     chunk slot and head (slots = T_total / 64 + N + 1) plus 128 KB per (sequence, head); e.g. 2
- *     sequences x 2048 tokens x 2 heads need 25.6 MiB.  Calls that need no workspace (fp32 q/k/v, dk
+ *     sequences x 2048 tokens x 2 heads need 21.5 MiB.  Calls that need no workspace (fp32 q/k/v, dk
  *     or dv = 64) have no limit.
  *   - Nothing in the scratch has to start at zero: every part a call reads is written earlier in the
  *     same call.

@@ -125,10 +125,10 @@ def test_workspace_size_is_a_pure_host_function(lib):
     assert kda.kda_chunk_fwd_workspace_size(0, 1, 1, 128, 128) == 0
     assert lib.kda_chunk_fwd_workspace_size(-1, 1, 1, 128, 128, 64) == 0
     assert kda.kda_chunk_fwd_workspace_size(4096, 1, 1, 64, 64) == 0   # the fp32 / d=64 paths use none
-    # one 192 KB record per (chunk slot, head), slots = T / 64 + N + 1; then two fp32 128 x 128 states
+    # one 160.5 KB record per (chunk slot, head), slots = T / 64 + N + 1; then two fp32 128 x 128 states
     # per (sequence, head) for the scan's intra-sequence split
-    assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) == (512 + 2) * 32 * 196608 + 2 * 32 * 65536
-    assert kda.kda_chunk_fwd_workspace_size(1000, 3, 2, 128, 128) == (15 + 4) * 2 * 196608 + 2 * 6 * 65536
+    assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) == (512 + 2) * 32 * 164352 + 2 * 32 * 65536
+    assert kda.kda_chunk_fwd_workspace_size(1000, 3, 2, 128, 128) == (15 + 4) * 2 * 164352 + 2 * 6 * 65536
 
 
 def test_static_scratch_rejects_oversize_before_any_cuda_call(lib):
