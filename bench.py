@@ -40,7 +40,8 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 64 * (3 * 128 + 2 * 128)
 # Decode: the fp32 state read and written once, plus q, k, v bf16, log_alpha fp32, beta fp32, o bf16.
 DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
-# The prefill with a workspace is two launches: the chunk-local kernel over every chunk, then the scan.
+# The prefill with a workspace is two launches for this workload: the chunk-local kernel over every
+# chunk, then the scan (calls with at most 8 (sequence, head) units add the scan's state-only pass).
 PREFILL_KERNELS_PER_CALL = 2
 PREFILL_KERNEL_SOURCES = ["gated_delta_rule_127_b200/csrc/kda_chunk_prep.cu",
                           "gated_delta_rule_127_b200/csrc/kda_chunk_scan.cu",
