@@ -268,3 +268,40 @@ def test_split_with_aliased_state():
     o, sf = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, state, inp.cu_seqlens,
                               final_state=state, dtype_o=torch.float32)
     assert torch.equal(o, o_ref) and torch.equal(state, s_ref)
+
+
+# ---------------------------------------------------------------- degenerate decay and write strength
+
+def _with_gates(inp, log_alpha_value=None, beta_value=None):
+    if log_alpha_value is not None:
+        inp.log_alpha = torch.full_like(inp.log_alpha, log_alpha_value)
+    if beta_value is not None:
+        inp.beta = torch.full_like(inp.beta, beta_value)
+    return inp
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+@pytest.mark.parametrize("case", ["no_decay", "beta_zero", "beta_one", "strong_decay_in_range"])
+def test_degenerate_gates(dtype, d, case):
+    """alpha = 1 (log_alpha = 0: the plain delta rule), beta = 0 (pure decay), beta = 1 (full
+    overwrite), and a decay whose cumulative log over a chunk reaches 76.8 nats on each side of the
+    anchor row -- inside the tensor-core path's 80-nat range -- all against the oracle."""
+    inp = gen.make_prefill([200, 64, 129], 2, d, d, dtype=dtype, init_state=True, seed=27, device=DEV)
+    la = {"no_decay": 0.0, "strong_decay_in_range": -2.4}.get(case)
+    b = {"beta_zero": 0.0, "beta_one": 1.0}.get(case)
+    _check_full(_with_gates(inp, la, b), dtype)
+
+
+def test_decay_beyond_the_anchor_range():
+    """log_alpha = -5 per token: the cumulative decay spans 160 nats on either side of a chunk's anchor.
+    The tf32 tensor-core path flags the chunks (KDA_DEVFLAG_DECAY_RANGE) instead of returning silently;
+    the fp32 path evaluates those chunks exactly and matches the oracle."""
+    inp = _with_gates(gen.make_prefill([300], 2, 128, 128, init_state=True, seed=28, device=DEV), -5.0)
+    kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, inp.cu_seqlens,
+                      dtype_o=torch.float32)
+    st, flags = kda.kda_get_device_status()
+    assert st == kda.KDA_ERR_DEVICE_CHECK and flags & kda.KDA_DEVFLAG_DECAY_RANGE
+    assert kda.kda_get_device_status() == (kda.KDA_OK, 0)
+    inp32 = _with_gates(gen.make_prefill([300], 2, 128, 128, dtype=torch.float32, init_state=True, seed=28,
+                                         device=DEV), -5.0)
+    _check_full(inp32, torch.float32)
