@@ -31,7 +31,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_max_over_ranks():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of this (multi-threaded) process
     mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
     assert out[0] == out[1] == 15.0
 
