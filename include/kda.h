@@ -98,7 +98,7 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int d
  * Path: dtype_qkv == KDA_FP32 runs the fp32 CUDA-core path (every product in fp32; no workspace
  * used).  KDA_BF16 with dk = dv = 128 runs on the tensor cores (tf32 products, fp32 accumulation and
  * fp32 state): with the workspace, a chunk-local kernel over all chunks at once followed by a scan
- * over each sequence's chunks (about 3 KB of workspace per token and head); without it, one kernel
+ * over each sequence's chunks (about 2.5 KB of workspace per token and head); without it, one kernel
  * per (sequence, head, 32-column slice of dv) that does both, slower.
  */
 KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
