@@ -584,8 +584,7 @@ cudaError_t launch_typed(const ChunkArgs& a) {
 }  // namespace
 
 bool chunk_tc_supported(const ChunkArgs& a) {
-    // T_total = 0 has no tile to describe; the CUDA-core path passes the states through.
-    return a.dtype_qkv == KDA_BF16 && a.dk == DK && a.dv == DV && a.T_total > 0 && a.T_total < (int64_t(1) << 31);
+    return chunk_tc_path(a.T_total, a.dtype_qkv, a.dk, a.dv);
 }
 
 template <bool SG>

@@ -55,6 +55,13 @@ struct DecodeArgs {
     float norm_eps;
 };
 
+// The bf16 dk = dv = 128 tensor-core prefill runs exactly when this holds; it is the only prefill
+// path that reads a workspace (T_total = 0 has no tile to describe and goes to the CUDA-core path,
+// which passes the states through).
+inline bool chunk_tc_path(int64_t T_total, kda_dtype dtype_qkv, int dk, int dv) {
+    return dtype_qkv == KDA_BF16 && dk == 128 && dv == 128 && T_total > 0 && T_total < (int64_t(1) << 31);
+}
+
 // Each launcher returns cudaSuccess or the launch error.
 cudaError_t launch_decode(const DecodeArgs& a);
 cudaError_t launch_chunk_simt(const ChunkArgs& a);

@@ -46,7 +46,11 @@ kda_status kda_chunk_fwd_static_scratch(const void* q, const void* k, const void
                                         int64_t T_total, int N, int H, int dk, int dv, int chunk_size,
                                         kda_dtype dtype_qkv, kda_dtype dtype_gate, kda_dtype dtype_o, void* o,
                                         float* final_state, void* stream) {
-    const size_t need = kda_chunk_fwd_workspace_size(T_total, N, H, dk, dv, chunk_size);
+    // Only the tensor-core path reads scratch; every other call (fp32 q/k/v, dk or dv = 64, no tokens)
+    // needs none and has no size limit.  The same predicate picks the path in kda_chunk_fwd.
+    const size_t need = kda::chunk_tc_path(T_total, dtype_qkv, dk, dv)
+                            ? kda_chunk_fwd_workspace_size(T_total, N, H, dk, dv, chunk_size)
+                            : 0;
     if (need > KDA_STATIC_SCRATCH_BYTES) return KDA_ERR_UNSUPPORTED;  // checked before any CUDA call
     void* scratch = nullptr;
     if (need > 0 && kda::static_scratch_ptr(&scratch) != cudaSuccess) return KDA_ERR_CUDA;

@@ -115,15 +115,19 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
 /*
  * kda_chunk_fwd for callers that cannot allocate device memory: the same arguments without the
  * workspace, the same results (the same kernels run).  The pages have no counterpart to this entry
- * point; it only changes where the scratch lives.  It allocates nothing: its scratch is a
- * file-scope device array of KDA_STATIC_SCRATCH_BYTES, reserved on a device when the library's
- * device code is loaded there, whose address is looked up once per device on the first call made
- * with that device current.
- *   - Limit: calls whose kda_chunk_fwd_workspace_size(...) exceeds KDA_STATIC_SCRATCH_BYTES return
- *     KDA_ERR_UNSUPPORTED before any CUDA call.  The size is one 160.5 KB chunk record per 64-token
- *     chunk slot and head (slots = T_total / 64 + N + 1) plus 128 KB per (sequence, head); e.g. 2
- *     sequences x 2048 tokens x 2 heads need 21.5 MiB.  Calls that need no workspace (fp32 q/k/v, dk
- *     or dv = 64) have no limit.
+ * point; it only changes where the scratch lives.  It allocates nothing itself: its scratch is a
+ * file-scope device array of KDA_STATIC_SCRATCH_BYTES, whose address is looked up once per device
+ * on the first call made with that device current.
+ *   - The array belongs to the library's device code, which CUDA loads onto a device lazily (by
+ *     default): the first call on a device that uses the array (one that runs on the tensor cores,
+ *     see the limit below) is when its 32 MiB get reserved there, and that call returns KDA_ERR_CUDA
+ *     if the device has no room left.  One small such call made once at set-up settles this early.
+ *   - Limit: a call that runs on the tensor cores (bf16 q/k/v, dk = dv = 128, T_total > 0) and whose
+ *     kda_chunk_fwd_workspace_size(...) exceeds KDA_STATIC_SCRATCH_BYTES returns KDA_ERR_UNSUPPORTED
+ *     before any CUDA call.  The size is one 160.5 KB chunk record per 64-token chunk slot and head
+ *     (slots = T_total / 64 + N + 1) plus 128 KB per (sequence, head); e.g. 2 sequences x 2048
+ *     tokens x 2 heads need 21.5 MiB.  Every other call (fp32 q/k/v, dk or dv = 64) reads no scratch
+ *     and has no limit, whatever kda_chunk_fwd_workspace_size says for its sizes.
  *   - Nothing in the scratch has to start at zero: every part a call reads is written earlier in the
  *     same call.
  *   - Every call on a device shares the one array: two calls that can run at the same time (on

@@ -139,6 +139,15 @@ def test_static_scratch_rejects_oversize_before_any_cuda_call(lib):
     assert st == kda.KDA_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("dq,d", [(kda.KDA_FP32, 128), (kda.KDA_BF16, 64)])
+def test_static_scratch_has_no_limit_off_the_tensor_core_path(lib, dq, d):
+    # the same oversize token count, but the call runs on the CUDA cores and reads no scratch: it gets
+    # past the size check and is rejected by kda_chunk_fwd's own validation (no output pointer) instead
+    st = lib.kda_chunk_fwd_static_scratch(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 65536, 1, 4, d, d, 64,
+                                          dq, kda.KDA_FP32, kda.KDA_FP32, None, None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+
+
 def test_ex_entry_points_reject_unknown_options_on_host(lib):
     ex = lambda opts, la=FAKE, g=None, w=None, eps=0.0: lib.kda_chunk_fwd_ex(
         FAKE, FAKE, FAKE, la, FAKE, None, None, 128, 1, 2, 128, 128, 64, kda.KDA_BF16, kda.KDA_FP32, kda.KDA_FP32,

@@ -49,6 +49,16 @@ def test_static_scratch_paths_without_workspace():
     assert torch.equal(s, s_ref)
 
 
+def test_static_scratch_fp32_beyond_the_nominal_size():
+    # fp32 q/k/v with dk = dv = 128: kda_chunk_fwd_workspace_size reports over 32 MiB for these sizes, but the
+    # call runs on the CUDA cores, reads no scratch and so has no limit
+    inp = gen.make_prefill([64] * 130, 2, 128, 128, dtype=torch.float32, init_state=True, seed=35, device=DEV)
+    assert kda.kda_chunk_fwd_workspace_size(inp.T_total, inp.N, 2, 128, 128) > 32 << 20
+    o, s, o_ref, s_ref = _both(inp)
+    assert torch.equal(o, o_ref)
+    assert torch.equal(s, s_ref)
+
+
 def test_static_scratch_rejects_oversize():
     inp = gen.make_prefill([65536], 4, 128, 128, dtype=torch.bfloat16, init_state=False, seed=34, device=DEV)
     with pytest.raises(kda.KdaError) as e:
