@@ -101,14 +101,12 @@ kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* lo
 
     cudaError_t err;
     bool epilogue_fused = false;
-    if (!chunk_tc_supported(a)) {
-        err = launch_chunk_simt(a);
-    } else if (have_ws && need > 0) {
+    if (chunk_tc_path(a.T_total, a.dtype_qkv, a.dk, a.dv) && have_ws && need > 0) {
         err = launch_chunk_prep(a);
         if (err == cudaSuccess) err = launch_chunk_scan(a);  // the scan applies the epilogue itself
         epilogue_fused = true;
-    } else {
-        err = launch_chunk_tc(a);
+    } else {  // fp32, d = 64, no tokens, or no workspace: the CUDA-core path
+        err = launch_chunk_simt(a);
     }
     if (err == cudaSuccess && a.epilogue && !epilogue_fused) err = launch_output_epilogue(a);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;

@@ -5,38 +5,54 @@
 // Chunk algorithm of "Kimi Linear: 표현력과 효율을 높인 어텐션 아키텍처(2025)", section "청크 단위
 // 병렬 알고리듬": cumulative log-decay inside the chunk, the beta-scaled decayed K K^T strictly lower
 // tile A, T = (I + A)^{-1} by forward substitution (the UT transform), and the WY factors
-// W = T Diag(beta) (K e^G), U = T Diag(beta) V.  With g = cumulative log-decay from the chunk start,
-// m = 32 the anchor row and Kt = K e^{g_C - G}:
-//   K+ = K e^{G - g_m},  Q+ = Q e^{G - g_m},  K- = K e^{g_m - G}         elementwise, fp32
-//   [A_raw; P] = [K+; Q+] (K-)^T                                         MMA 1 (A operand in TMEM)
-//   A = beta_r A_raw strictly lower, P lower with the diagonal
+// W = T Diag(beta) (K e^G), U = T Diag(beta) V.  With g the cumulative log-decay from the chunk start
+// and Kt = K e^{g_C - G}:
+//   A_ri = beta_r sum_c k_rc k_ic e^{g_rc - g_ic} (i < r),   P_ti = sum_c q_tc k_ic e^{g_tc - g_ic} (i <= t)
 //   T = (I + A)^{-1}: 16 x 16 diagonal blocks by forward substitution (fp32), then merged into
 //       32 x 32 and 64 x 64 inverses with [[T1, 0], [-T2 A21 T1, T2]] on warp-level tensor-core
 //       tiles (mma.sync tf32, fp32 accumulation)
-//   [W | U] = T [beta K e^G | beta V]                                    MMA 2
-//   B^T = U^T Kt,  Uo^T = U^T P^T (MMAs 5-6, first),  P W,  Kt^T W (MMAs 3-4)
-//   Mt = Diag(e^{g_C}) - Kt^T W,  Qh = Q e^G - P W
-// B and Uo are formed transposed so that the accumulator lane is the value column: they go from
-// registers straight to memory in contiguous runs.  Mt and Qh are staged in shared memory as the
-// scan's operand tiles and written with bulk copies.
-// The anchor split e^{g_r - g_i} = e^{g_r - g_m} e^{g_m - g_i} keeps every factor that can exceed 1
-// below e^80 while the chunk's log-decay stays within 80 of g_m at both ends ("일반 DPLR보다 줄어든
-// 연산량" on the same page notes that fine-grained decay makes intra-chunk division delicate);
-// outside that range the chunk sets KDA_DEVFLAG_DECAY_RANGE.  Every MMA runs kind::tf32 with fp32
-// accumulation (operands rounded to tf32 when written); B is stored in fp16 with a power-of-two
-// exponent per 32 rows and value column (fp16 keeps tf32's 10-bit mantissa), Uo in fp32.
+//   W^T = (beta K e^G)^T T^T,  U^T = (beta V)^T T^T                MMA 2 (A operands in tensor memory)
+//   [Mt^T - Diag(e^{g_C}) | Qh^T - (Q e^G)^T] = -W^T [Kt | P^T]      MMA 3 (N = 192)
+//   [B^T | Uo^T] = U^T [Kt | P^T]                                    MMA 4 (N = 192)
+// Everything is formed transposed, with the key channel (or value column) as the tensor-memory lane:
+// the elementwise pass owns a channel and writes its operands straight into tensor memory, and each
+// record row goes from a lane's registers to the record in coalesced runs.  Every tcgen05 tf32 MMA
+// instruction costs about the same time for any N up to 192, so the products are grouped into few
+// wide instructions: 16 for MMA 1, 16 for MMA 2, 8 each for MMAs 3 and 4.
 //
-// Persistent CTAs of 512 threads, one per SM, each taking (chunk slot, head) tasks in turn.  The next
-// task's input tiles are loaded into shared memory while the task's results are being stored.
-// Elementwise pass: thread t owns key channel c = 32 (w % 4) + lane (its tensor-memory lane, w =
-// warp) and rows 16 (w / 4) .. +15, so the cumulative sum runs down a column in registers.  Row pass
-// and accumulator read-outs: the warp's lane quadrant gives the row, w / 4 the column quarter (M = 64
-// accumulators through the 16x32bx2 shape, lanes 16..31 taking a second column range).
+// Decay factors: secondary chunking.  "일반 DPLR보다 줄어든 연산량" on the same page notes that with a
+// decay per channel the intra-chunk division is numerically delicate (a factor e^{-g} overflows) and
+// points to the log domain with a second level of chunking.  Each chunk is cut into four 16-row
+// blocks; row block R has one anchor a_R per channel, and
+//   e^{g_r - g_i} = e^{g_r - a_R} e^{a_R - g_i}        for r in block R and i up to the block's last row.
+// For i in an earlier block both factors are <= 1 whatever the decay (a_R is at most g at the
+// block's first row, which is at most g_i).  Inside the block a_R is the midpoint of the channel's
+// log-decay across the block, so both factors stay <= e^{span / 2} <= e^40 while that span is at
+// most 80 nats.  A channel whose span is larger (strong decay, e.g. 20 nats a token) takes a_R = g
+// at the block's first row instead, is left out of the block's diagonal 16 x 16 product, and its
+// diagonal terms are added one by one with the exact e^{g_r - g_i}.  No factor exceeds e^40 and
+// every factor that underflows multiplies a true value at least as small, so every chunk is exact up
+// to rounding for every alpha in (0, 1).  MMA 1 is one MMA with N = 160: the [K; Q] rows scaled by
+// e^{G - a} (A operand in tensor memory) against the column tiles K e^{a_R - G} of all four blocks
+// stacked (16 + 32 + 48 + 64 rows); row r of block R keeps the columns of tile R.
+//
+// Persistent CTAs of 512 threads, one per SM, each taking (chunk slot, head) tasks in turn; the next
+// task's input tiles are loaded while the current task runs its inverse and products, and the
+// record's Mt and Qh tiles leave through bulk copies while the next task starts.  Elementwise pass:
+// thread t owns key channel c = 32 (w % 4) + lane (its tensor-memory lane, w = warp) and rows
+// 16 I + 4 (w / 4) .. + 3 of every block I (a cumulative sum over 4-row groups, completed through
+// shared memory).  Row pass and read-outs: the warp's lane quadrant gives the row (or channel),
+// w / 4 the column quarter.
+// Every MMA runs kind::tf32 with fp32 accumulation (operands rounded to tf32 when written); B is
+// stored in fp16 with a power-of-two exponent per 32 rows and value column (fp16 keeps tf32's
+// 10-bit mantissa), Uo in fp32.
 // Template options: TG the gate dtype; SG Gated DeltaNet's scalar gate (one rate per token and head,
 // read with beta, broadcast over the channels in the cumulative sum); PRO the fused L2 normalisation
 // of q and k (each use of a row scaled by 1 / its norm).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <type_traits>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -54,58 +70,96 @@ using wy::DV;
 
 constexpr int THREADS = 512;
 constexpr int TP = 68;  // row stride (floats) of the fp32 A and T tiles (conflict-free MMA fragment reads)
-constexpr float kAnchorLimit = 80.f;
+constexpr float kSpanLimit = 80.f;  // largest log-decay span of a 16-row block kept in its MMA product
 constexpr uint32_t kWaitPolls = 1u << 26;
 
-// ---- shared memory (bytes from a 1024-aligned base); later phases reuse regions that are dead
+// ---- shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_SQ = 0;         // q staging bf16 [64][128], two 64-channel boxes, 128-byte swizzle
-constexpr uint32_t OFF_G = 16384;      // log_alpha staging; then E = e^{G - g_m} fp32, sw128_off(r, c, 64)
-constexpr uint32_t OFF_SK = 49152;     // k staging bf16
-constexpr uint32_t OFF_SV = 65536;     // v staging bf16
-constexpr uint32_t OFF_KM = 81920;     // K- K-major: rows s (64) x K c (128), MMA 1's B
-constexpr uint32_t OFF_B8 = 114688;    // [beta K e^G | beta V] K-major: rows n (256) x K s (64), MMA 2's B;
-                                       //   then [W | U] MN-major: K-rows s (64) x N n (256), operand of MMAs 3-6
-constexpr uint32_t OFF_KT = 180224;    // Kt^T K-major: rows c (128) x K s (64), A of MMA 4 and B of MMA 5
-constexpr uint32_t OFF_MISC = 212992;  // beta[2][64] (this task, the next), quarter-column sums[4][128],
-                                       //   g_m, g_C, e^{g_m}, e^{g_C} [128]
-constexpr uint32_t OFF_X = 217600;     // 32 x 32 fp32 scratch for the inverse
-constexpr uint32_t OFF_TASK = 221696;  // three Task slots (this task, the next, the one after)
-constexpr uint32_t OFF_BARS = 221792;  // mbarriers: TMA, MMAs 1-2, MMAs 3-4, MMAs 5-6; then the TMEM base address
-constexpr uint32_t OFF_SAL = 221840;   // scalar log-decay [2][64] (Gated DeltaNet gates), by task parity
-constexpr uint32_t OFF_RN = OFF_SAL + 512;  // 1 / ||k_r|| [64], 1 / ||q_r|| [64] (fused L2 normalisation)
+constexpr uint32_t OFF_SK = 16384;     // k staging bf16
+constexpr uint32_t OFF_SV = 32768;     // v staging bf16; later P in fp32 while strong-decay terms are added
+constexpr uint32_t OFF_G = 49152;      // log_alpha staging; then, fp32 at sw128_off(r, c, 64), the row factors
+                                       //   e^{g - a} -- or g itself when some channel decays strongly
+constexpr uint32_t OFF_Y = 81920;      // column tiles of MMA 1: tile R (rows 0 .. 16 R + 15, K e^{a_R - G}) at rows
+                                       //   y_row(R) .. of one K-major tile, 160 rows x K c (128), sw128_off(n, c, 160)
+constexpr uint32_t OFF_KP = 163840;    // [Kt; P] K-major: rows n (Kt^T rows c 0..127, P rows t 128..191) x K s (64),
+                                       //   sw128_off(n, s, 192): B of MMAs 3 and 4
+// per-channel factors of each 16-row block, until P is written over them (the P rows of each K-block):
+constexpr uint32_t OFF_FAC = OFF_KP + 16384;   // anchors a[4][128], e^{g_e - a}[4][128], e^{g_C - g_e}[4][128],
+                                               //   e^{a}[4][128]  (g_e: g at the block's last row)
+constexpr uint32_t OFF_RHO = OFF_KP + 40960;   // e^{a_R - g_eI} [6][128] for block pairs R > I
+constexpr uint32_t OFF_XP = 212992;    // column sums of each 4-row group [16][128]
+constexpr uint32_t OFF_MISC = 221184;  // beta[2][64] (this task, the next), e^{g_C} [128], strong-decay channel
+                                       //   masks [4 blocks][4 words]
+constexpr uint32_t MISC_BYTES = (128 + 128) * 4 + 64;
+constexpr uint32_t OFF_TASK = OFF_MISC + MISC_BYTES;  // three Task slots (this task, the next, the one after)
+constexpr uint32_t OFF_BARS = OFF_TASK + 96;   // mbarriers: TMA, MMA 1, MMA 2, MMA 3, MMA 4; then the TMEM base
+constexpr uint32_t OFF_SAL = OFF_BARS + 48;    // scalar log-decay [2][64] (Gated DeltaNet gates), by task parity
+constexpr uint32_t OFF_RN = OFF_SAL + 512;     // 1 / ||k_r|| [64], 1 / ||q_r|| [64] (fused L2 normalisation)
 constexpr uint32_t SMEM_USED = OFF_RN + 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
-// after MMA 1 (k, v staging and K- are dead):
-constexpr uint32_t OFF_A = 49152;      // A fp32 [64][TP]
-constexpr uint32_t OFF_T32 = 66560;    // T fp32 [64][TP]
-constexpr uint32_t OFF_TIMG = 49152;   // T K-major rows r x K s (64), MMA 2's A (over A, once T is formed)
-constexpr uint32_t OFF_P = 84992;      // P K-major rows t x K s (64), A of MMA 3 and B of MMA 6
-// record staging once MMAs 3-6 are done, outside the input staging so the next task's tiles can load:
-constexpr uint32_t STG_M = OFF_B8;     // Mt K-major rows i x K j (128), 64 KB
-constexpr uint32_t STG_Q = OFF_KT;     // Qh K-major rows t x K j (128), 32 KB
+// after MMA 1 (the column tiles are dead):
+constexpr uint32_t OFF_A = OFF_Y;              // A fp32 [64][TP]
+constexpr uint32_t OFF_T32 = OFF_Y + 17408;    // T fp32 [64][TP]
+constexpr uint32_t OFF_TIMG = OFF_Y + 35840;   // T K-major rows r x K s (64), B of MMA 2
+constexpr uint32_t OFF_XS = OFF_Y + 52224;     // 32 x 32 fp32 scratch for the inverse
+constexpr uint32_t OFF_PF = OFF_SV;            // P fp32 [64][64] (16-byte chunks XOR-swizzled by row)
+// after MMA 2:
+constexpr uint32_t OFF_WT = OFF_Y;             // -W^T K-major rows j x K s (64), A of MMA 3
+constexpr uint32_t OFF_UT = OFF_Y + 32768;     // U^T K-major rows dv x K s (64), A of MMA 4
+// after MMAs 3 and 4: the record's Qh and Mt tiles, in the record's layout, for two bulk copies
+constexpr uint32_t OFF_STQ = OFF_Y;            // Qh, 32 KB
+constexpr uint32_t OFF_STM = OFF_Y + 32768;    // Mt, 64 KB
+static_assert(OFF_STM + 65536 <= OFF_XP, "record staging");
+static_assert(OFF_XS + 4096 <= OFF_KP && OFF_UT + 32768 <= OFF_KP, "tiles overlap [Kt; P]");
+static_assert(OFF_XP + 16 * 128 * 4 <= OFF_MISC, "group sums");
+static_assert(OFF_FAC + 16 * 128 * 4 <= OFF_KP + 24576 && OFF_RHO + 6 * 128 * 4 <= OFF_KP + 49152, "factors");
+static_assert(OFF_KP + 49152 <= OFF_XP, "[Kt; P]");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(OFF_TIMG % 1024 == 0 && OFF_WT % 1024 == 0 && OFF_UT % 1024 == 0 && OFF_Y % 1024 == 0 &&
+              OFF_KP % 1024 == 0, "swizzle atoms");
+
+// first row of column tile R within the 160-row tile (tile R has 16 R + 16 rows)
+__host__ __device__ constexpr int y_row(int R) { return 8 * R * (R + 1); }
+// index of the block pair (R, I), R > I, in OFF_RHO
+__host__ __device__ constexpr int rho_idx(int R, int I) { return R * (R - 1) / 2 + I; }
 
 // ---- tensor memory columns (512 allocated)
-constexpr uint32_t TM_A1 = 0;     // [K+; Q+], 128 x 128, MMA 1's A
-constexpr uint32_t TM_D1 = 128;   // [A_raw; P], 128 x 64
-constexpr uint32_t TM_D8 = 256;   // [W | U], M=64 layout, 256 columns
-constexpr uint32_t TM_PW = 0;     // P W, M=64 layout, 128 columns          (after [W | U] is read out)
-constexpr uint32_t TM_KW = 128;   // Kt^T W, 128 x 128
-constexpr uint32_t TM_BT = 256;   // B^T = U^T Kt, 128 (dv) x 128 (i)
-constexpr uint32_t TM_UT = 384;   // Uo^T = U^T P^T, 128 (dv) x 64 (t)
+constexpr uint32_t TM_X = 0;      // [K; Q] rows scaled by e^{G - a}, 128 x 128, A of MMA 1
+constexpr uint32_t TM_D1 = 128;   // MMA 1, 128 x 160: block R's columns at TM_D1 + y_row(R)
+constexpr uint32_t TM_BK = 320;   // (beta K e^G)^T, 128 (c) x 64 (s), A of MMA 2
+constexpr uint32_t TM_BV = 384;   // (beta V)^T, 128 (dv) x 64 (s), A of MMA 2
+constexpr uint32_t TM_QG = 448;   // (Q e^G)^T, 128 (j) x 64 (t): added to Qh^T when it is read out
+constexpr uint32_t TM_WT = 0;     // W^T, 128 x 64 (after MMA 1)
+constexpr uint32_t TM_UT = 64;    // U^T, 128 x 64
+constexpr uint32_t TM_DW = 0;     // MMA 3, 128 (j) x 192: -W^T Kt (i = 0..127), then -W^T P^T (t)   (after MMA 2)
+constexpr uint32_t TM_DU = 192;   // MMA 4, 128 (dv) x 192: B^T = U^T Kt, then Uo^T = U^T P^T
 constexpr uint32_t TM_COLS = 512;
+
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// 1 / x (the MUFU approximation, within an ulp or two of fp32; every use rounds to tf32 afterwards)
+__device__ __forceinline__ float recip_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Byte offset of element (t, i) of the fp32 P tile at OFF_PF: rows of 256 bytes, 16-byte chunk i / 4
+// XOR-swizzled with t % 16 so that a warp's rows do not share banks.
+__device__ __forceinline__ uint32_t pf_off(int t, int i) {
+    return static_cast<uint32_t>(t * 256 + ((((i >> 2) ^ (t & 15))) << 4) + ((i & 3) << 2));
+}
 
 // Byte offset of element (r, c) of a bf16 [64][128] tile loaded as two 64-channel boxes with the
 // 128-byte swizzle: box c / 64, row r at r * 128, 16-byte chunks permuted by XOR with r % 8.
 __device__ __forceinline__ uint32_t bf16_sw_off(int r, int c) {
     return static_cast<uint32_t>((c >> 6) * 8192 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
-}
-
-template <typename TG> __device__ __forceinline__ float gate_at(const unsigned char* sm, int r, int c);
-template <> __device__ __forceinline__ float gate_at<float>(const unsigned char* sm, int r, int c) {
-    return *reinterpret_cast<const float*>(sm + OFF_G + sw128_off(r, c, 64));
-}
-template <> __device__ __forceinline__ float gate_at<__nv_bfloat16>(const unsigned char* sm, int r, int c) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_G + 16384 + bf16_sw_off(r, c)));
 }
 
 __device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {
@@ -117,13 +171,6 @@ __device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {
     }
 }
 
-__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // Task = (chunk slot, head), slot-major so consecutive tasks share the same tokens.
 struct Task {
@@ -286,6 +333,7 @@ __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, f
     __syncthreads();
 }
 
+
 // SG: Gated DeltaNet gates -- log_alpha is [T_total, H], one decay rate per token and head, read
 // with beta and broadcast over the key channels (tm_g is then unused).
 // PRO: q and k arrive raw; every use of a row is scaled by 1 / its L2 norm, computed per chunk.
@@ -298,27 +346,31 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   unsigned char* __restrict__ ws, unsigned int* flags, int beta_logits) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;   // tensor-memory lane quadrant
-    const int qr = warp >> 2;  // row quarter (elementwise pass) / column quarter (read-outs)
+    const int qr = warp >> 2;  // row block (elementwise pass) / column quarter (row pass, read-outs)
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(sm);
     float* s_beta2 = reinterpret_cast<float*>(sm + OFF_MISC);  // [2][64], by task parity
-    float* x_part = s_beta2 + 128;  // [4][128]
-    float* x_gm = x_part + 512;
-    float* x_gc = x_gm + 128;
-    float* x_egm = x_gc + 128;
-    float* x_gam = x_egm + 128;
+    float* s_gam = s_beta2 + 128;   // [128] e^{g_C}
+    uint32_t* s_strong = reinterpret_cast<uint32_t*>(s_gam + 128);  // [4 blocks][4 words] strong-decay channels
+    float* x_part = reinterpret_cast<float*>(sm + OFF_XP);     // [16 groups][128]
+    float* f_anc = reinterpret_cast<float*>(sm + OFF_FAC);     // [4][128] anchors
+    float* f_tau = f_anc + 512;     // [4][128] e^{g_e - a}
+    float* f_kap = f_tau + 512;     // [4][128] e^{g_C - g_e}
+    float* f_ea = f_kap + 512;      // [4][128] e^{a}
+    float* f_rho = reinterpret_cast<float*>(sm + OFF_RHO);     // [6][128] e^{a_R - g_eI}
     float* s_alpha2 = reinterpret_cast<float*>(sm + OFF_SAL);  // [2][64] (SG only)
     float* s_rn = reinterpret_cast<float*>(sm + OFF_RN);       // [128]: k rows, then q rows (PRO only)
-    float* xs = reinterpret_cast<float*>(sm + OFF_X);
+    float* xs = reinterpret_cast<float*>(sm + OFF_XS);
     Task* slots = reinterpret_cast<Task*>(sm + OFF_TASK);  // ring of 3: this task, the next, the one after
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
-    uint64_t* bar_mma = bar_tma + 1;   // MMAs 1 and 2
-    uint64_t* bar_rest = bar_tma + 2;  // MMAs 3-4
-    uint64_t* bar_bu = bar_tma + 3;    // MMAs 5-6
-    uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 32);
+    uint64_t* bar_m1 = bar_tma + 1;
+    uint64_t* bar_m2 = bar_tma + 2;
+    uint64_t* bar_m3 = bar_tma + 3;
+    uint64_t* bar_m4 = bar_tma + 4;
+    uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 40);
 
     constexpr uint32_t kGateBytes = SG ? 0 : C * DK * sizeof(TG);
     constexpr uint32_t kStageBytes = 3 * C * DK * 2 + kGateBytes;
@@ -342,10 +394,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         slots[2].id = -1;
     }
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(bar_mma, 1);
-        mbar_init(bar_rest, 1);
-        mbar_init(bar_bu, 1);
+        for (int b = 0; b < 5; ++b) mbar_init(bar_tma + b, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
         if (!SG) tma_prefetch_desc(&tm_g);
@@ -376,6 +425,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     load_beta(slots[0], 0);  // (slots are written by thread 0 before the barrier above)
     __syncthreads();
 
+    const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK);
+    const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ);
+    auto gf_at = [&](int r, int ch) -> float& { return *reinterpret_cast<float*>(sm + OFF_G + sw128_off(r, ch, 64)); };
+    const int rbq = 4 * qr;  // the elementwise pass's rows: 16 I + rbq .. + 3 of every block I
+    // Byte offsets of (row, channel c) within a 128-byte row, for rows congruent to rbq + w mod 8: swf[w]
+    // in the fp32 tiles (sw128_off), swb[w] in the bf16 staging tiles (bf16_sw_off, block of 64 channels
+    // included); sw*0 for rows congruent to 0.
+    uint32_t swf[4], swb[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t x = static_cast<uint32_t>((rbq + w) & 7);
+        swf[w] = ((static_cast<uint32_t>(lane >> 2) ^ x) << 4) | (static_cast<uint32_t>(lane & 3) << 2);
+        swb[w] = static_cast<uint32_t>(q4 >> 1) * 8192u +
+                 ((static_cast<uint32_t>(4 * (q4 & 1) + (lane >> 3)) ^ x) << 4) + (static_cast<uint32_t>(lane & 7) << 1);
+    }
+    const uint32_t swf0 = (static_cast<uint32_t>(lane >> 2) << 4) | (static_cast<uint32_t>(lane & 3) << 2);
+    const uint32_t swb0 = static_cast<uint32_t>(q4 >> 1) * 8192u + (static_cast<uint32_t>(4 * (q4 & 1) + (lane >> 3)) << 4) +
+                          (static_cast<uint32_t>(lane & 7) << 1);
+    const uint32_t colf = static_cast<uint32_t>(q4) * 8192u;  // channel block of c in a 64-row fp32 tile
+
     int cur = 0;  // slot of this task in the ring of three
     for (uint32_t it = 0;; ++it, cur = cur == 2 ? 0 : cur + 1) {  // `it`: tasks taken; phase parities follow from it
         const int nxt = cur == 2 ? 0 : cur + 1, aft = nxt == 2 ? 0 : nxt + 1;
@@ -383,22 +452,35 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (tk.id < 0) break;
         const int len = tk.len;
         unsigned char* rec = tk.rec;
-        const float* s_beta = s_beta2 + 64 * (it & 1);
-        failed = !mbar_wait(bar_tma, it & 1, kWaitPolls);
+        const uint32_t par = it & 1;
+        const float* s_beta = s_beta2 + 64 * par;
+        failed = !mbar_wait(bar_tma, par, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
+        tc_fence_after_sync();
 
-        // ---- elementwise pass: cumulative log-decay down channel c, rows rb .. rb+15
-        const int rb = 16 * qr;
-        float g[16];
-        {
+        // ---- elementwise pass, 1: log-decays of channel c over rows 16 I + rbq .. + 3 of each block I; the
+        //      sum of each 4-row group goes to x_part[group]
+        // log-decay of row r of channel c, with the row's swizzle parts
+        auto a_at = [&](int r, uint32_t sf, uint32_t sb) -> float {
+            if (r >= len) return 0.f;
+            if (SG) return s_alpha2[64 * par + r];
+            if (sizeof(TG) == 4) return *reinterpret_cast<const float*>(sm + OFF_G + colf + r * 128 + sf);
+            return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_G + 16384 + sb + r * 128));
+        };
+        float g[4][4];
+#pragma unroll
+        for (int I = 0; I < 4; ++I) {
             float run = 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                run += (rb + r) < len ? (SG ? s_alpha2[64 * (it & 1) + rb + r] : gate_at<TG>(sm, rb + r, c)) : 0.f;
-                g[r] = run;
+            for (int w = 0; w < 4; ++w) {
+                run += a_at(16 * I + rbq + w, swf[w], swb[w]);
+                g[I][w] = run;
             }
-            x_part[qr * 128 + c] = run;
+            x_part[(4 * I + qr) * 128 + c] = run;
         }
+        float a_first[4];  // log-decay of each block's first row (the thread with rbq = 0 holds it as g[I][0])
+#pragma unroll
+        for (int I = 0; I < 4; ++I) a_first[I] = a_at(16 * I, swf0, swb0);
         if (PRO) {  // 1 / ||k_r|| and 1 / ||q_r||: warp w takes rows 8 w .. 8 w + 7 of [K; Q], 4 channels a lane
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -413,54 +495,116 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
         __syncthreads();
+        // ---- 2: g from the chunk start; every block's first and last g, anchor and strong-decay flag for
+        //      channel c (the four threads of a channel compute the same; those with qr = 0 publish them)
+        float anc[4], gl[4];
+        uint32_t strong = 0;  // bit I: block I's span exceeds kSpanLimit
         {
             float off = 0.f;
-            for (int q = 0; q < qr; ++q) off += x_part[q * 128 + c];
+            float gfst[4];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) g[r] += off;
-            if (qr == 2) { x_gm[c] = g[0]; x_egm[c] = expf(g[0]); }     // row 32
-            if (qr == 3) { x_gc[c] = g[15]; x_gam[c] = expf(g[15]); }   // row 63 (padded rows add nothing)
-        }
-        if (tid == 0) bulk_wait_read();  // the previous record has left the Mt and Qh staging tiles
-        __syncthreads();
-        {
-            const float gm = x_gm[c], gC = x_gc[c], egm = x_egm[c];
-            const float ecm = __expf(gC - gm);
-            if ((qr == 0 && g[0] - gm > kAnchorLimit) || (qr == 3 && gm - gC > kAnchorLimit))
-                raise_flag(flags, KDA_DEVFLAG_DECAY_RANGE);
-            const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK);
-            const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SV);
+            for (int G = 0; G < 16; ++G) {
+                const int I = G >> 2;
+                if ((G & 3) == 0) gfst[I] = off + a_first[I];
+                if ((G & 3) == qr) {
 #pragma unroll
-            for (int r4 = 0; r4 < 16; r4 += 4) {
-                float kt[4], bk[4], bv[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int R = rb + r4 + u;
-                    const bool live = R < len;
-                    const float kv = live ? __bfloat162float(sk[bf16_sw_off(R, c) >> 1]) * (PRO ? s_rn[R] : 1.f) : 0.f;
-                    const float vv = live ? __bfloat162float(sv[bf16_sw_off(R, c) >> 1]) : 0.f;
-                    const float b = s_beta[R];
-                    const float e = __expf(g[r4 + u] - gm), ie = __expf(gm - g[r4 + u]);
-                    *reinterpret_cast<float*>(sm + OFF_G + sw128_off(R, c, 64)) = e;
-                    *reinterpret_cast<float*>(sm + OFF_KM + sw128_off(R, c, 64)) = to_tf32(kv * ie);
-                    kt[u] = to_tf32(kv * ie * ecm);
-                    bk[u] = to_tf32(b * kv * e * egm);
-                    bv[u] = to_tf32(b * vv);
+                    for (int w = 0; w < 4; ++w) g[I][w] += off;
                 }
-                const int R0 = rb + r4;
-                *reinterpret_cast<float4*>(sm + OFF_KT + sw128_off(c, R0, 128)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
-                *reinterpret_cast<float4*>(sm + OFF_B8 + sw128_off(c, R0, 256)) = make_float4(bk[0], bk[1], bk[2], bk[3]);
-                *reinterpret_cast<float4*>(sm + OFF_B8 + sw128_off(DK + c, R0, 256)) =
-                    make_float4(bv[0], bv[1], bv[2], bv[3]);
+                off += x_part[G * 128 + c];
+                if ((G & 3) == 3) gl[I] = off;
+            }
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+                const float span = gfst[I] - gl[I];  // >= 0: g does not increase down the chunk
+                const bool st = span > kSpanLimit;
+                strong |= st ? (1u << I) : 0u;
+                anc[I] = st ? gfst[I] : gfst[I] - 0.5f * span;
+            }
+            // block I = qr's factors for channel c (the four threads of the channel split the blocks)
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+                if (I != qr) continue;
+                f_anc[I * 128 + c] = anc[I];
+                f_tau[I * 128 + c] = __expf(gl[I] - anc[I]);
+                f_kap[I * 128 + c] = __expf(gl[3] - gl[I]);
+                f_ea[I * 128 + c] = __expf(anc[I]);
+#pragma unroll
+                for (int R = I + 1; R < 4; ++R) f_rho[rho_idx(R, I) * 128 + c] = __expf(anc[R] - gl[I]);
+                const uint32_t m = __ballot_sync(0xffffffffu, (strong >> I) & 1u);
+                if (lane == 0) s_strong[I * 4 + q4] = m;
+                if (I == 3) s_gam[c] = __expf(gl[3]);
             }
         }
+        if (tid == 0) bulk_wait_read();  // the previous record's Qh and Mt tiles have left shared memory
+        const bool any_strong = __syncthreads_or(strong != 0);
+
+        // ---- 3: per element (row i, channel c): the row factor e^{g_i - a} (for the row pass; g itself when
+        //      some channel decays strongly), the column tiles of MMA 1, Kt^T (MMAs 3-4), (beta K e^G)^T,
+        //      (beta V)^T (MMA 2) and (Q e^G)^T.  For i in block I, F_i = e^{g_eI - g_i} <= 1 (eI the block's
+        //      last row); diagonal column factor e^{a_I - g_i} (1 / the row factor); column factor of a later
+        //      block R: e^{a_R - g_eI} F_i (both <= 1)
+        auto elementwise = [&](auto full_chunk) {
+            constexpr bool kFull = decltype(full_chunk)::value;  // every row live: no masks
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+                const bool st = (strong >> I) & 1u;
+                const float tau = f_tau[I * 128 + c], kap = f_kap[I * 128 + c], ea = f_ea[I * 128 + c];
+                float rho[4];
+#pragma unroll
+                for (int R = I + 1; R < 4; ++R) rho[R] = f_rho[rho_idx(R, I) * 128 + c];
+                float kt[4], bk[4], bv[4], qg[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const int i = 16 * I + rbq + w;
+                    const bool live = kFull || i < len;
+                    const uint32_t ob = swb[w] + i * 128;  // (i, c) in the bf16 staging tiles
+                    float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK + ob));
+                    float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ + ob));
+                    float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SV + ob));
+                    if (PRO) { kv *= s_rn[i]; qv *= s_rn[64 + i]; }
+                    if (!live) { kv = 0.f; qv = 0.f; vv = 0.f; }
+                    const float b = s_beta[i];
+                    float dc, F, Gm, rowf;
+                    if (!st) {
+                        dc = __expf(anc[I] - g[I][w]);  // e^{a_I - g_i} in [e^-40, e^40]
+                        rowf = recip_approx(dc);        // e^{g_i - a_I}
+                        F = dc * tau;                   // >= e^-80: a normal float
+                        Gm = rowf * ea;                 // e^{g_i} (only values below e^-47 lose digits)
+                    } else {
+                        dc = 0.f;                       // left to the exact per-element terms
+                        rowf = 0.f;
+                        F = __expf(gl[I] - g[I][w]);
+                        Gm = __expf(g[I][w]);
+                    }
+                    *reinterpret_cast<float*>(sm + OFF_G + colf + i * 128 + swf[w]) = any_strong ? g[I][w] : rowf;
+                    // column tiles: (n, c) at q4 * 160 * 128 + n * 128 + swizzle, n = y_row(R) + i = i mod 8
+                    unsigned char* ycol = sm + OFF_Y + q4 * 20480 + swf[w] + i * 128;
+                    const float kf = kv * F;
+                    *reinterpret_cast<float*>(ycol + y_row(I) * 128) = to_tf32(kv * dc);
+#pragma unroll
+                    for (int R = I + 1; R < 4; ++R) *reinterpret_cast<float*>(ycol + y_row(R) * 128) = to_tf32(kf * rho[R]);
+                    kt[w] = to_tf32(kf * kap);
+                    bk[w] = to_tf32(b * kv * Gm);
+                    bv[w] = to_tf32(b * vv);
+                    qg[w] = qv * Gm;
+                }
+                *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 192)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+                tmem_st4(tq + TM_BK + 16 * I + rbq, bk);
+                tmem_st4(tq + TM_BV + 16 * I + rbq, bv);
+                tmem_st4(tq + TM_QG + 16 * I + rbq, qg);
+            }
+        };
+        if (len == C) elementwise(std::true_type{});
+        else elementwise(std::false_type{});
         __syncthreads();
 
-        // ---- row pass: [K+; Q+] into tensor memory (lane = row: 0..63 K+, 64..127 Q+), channels 32 qr ..
+        // ---- row pass: X = [K; Q] e^{G - a} into tensor memory (lane = row: 0..63 K, 64..127 Q; a the anchor
+        //      of the row's block), channels 32 qr ..
         {
-            const int r = c & 63;
-            const unsigned char* src = sm + (c < 64 ? OFF_SK : OFF_SQ);
-            const bool live = r < len;
+            const bool isq = c >= 64;
+            const int r = c & 63, R = r >> 4;
+            const unsigned char* src = sm + (isq ? OFF_SQ : OFF_SK);
+            const bool live = r < len;  // (len is the same for the whole CTA: no divergence when it is C)
             const int cb = 32 * qr;
             const float rn = PRO ? s_rn[c] : 1.f;  // lanes 0..63 k rows, 64..127 q rows
             float v[32];
@@ -469,59 +613,148 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int cc = cb + 8 * e8;
                 float x[8];
                 unpack8(*reinterpret_cast<const uint4*>(src + bf16_sw_off(r, cc)), x);
-                const float4 e0 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(r, cc, 64));
-                const float4 e1 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(r, cc + 4, 64));
-                const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                const float4 f0 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(r, cc, 64));
+                const float4 f1 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(r, cc + 4, 64));
+                float fv[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                if (any_strong) {  // the buffer holds g: the factor is e^{g - a} (<= e^40, or <= 1 where strong)
+                    const float4 a0 = *reinterpret_cast<const float4*>(f_anc + R * 128 + cc);
+                    const float4 a1 = *reinterpret_cast<const float4*>(f_anc + R * 128 + cc + 4);
+                    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[8 * e8 + i] = live ? to_tf32(x[i] * rn * ev[i]) : 0.f;
+                    for (int i = 0; i < 8; ++i) fv[i] = __expf(fv[i] - av[i]);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[8 * e8 + i] = to_tf32((PRO ? x[i] * rn : x[i]) * fv[i]);
+                if (!live) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[8 * e8 + i] = 0.f;
+                }
             }
-            tmem_st32(tq + TM_A1 + cb, v);
-            tmem_st_wait();
+            tmem_st32(tq + TM_X + cb, v);
         }
+        tmem_st_wait();
         fence_async_smem();
         tc_fence_before_sync();
         __syncthreads();
 
-        // ---- MMA 1: [A_raw; P] = [K+; Q+] (K-)^T   (M=128, N=64, K=128)
+        // ---- MMA 1: [A_raw; P] = X Y^T (M=128, N=160, K=128): row r of block R uses the columns of tile R
         if (tid == 0) {
             tc_fence_after_sync();
-            const uint64_t bkm = sw128_desc(sbase + OFF_KM, 16, 1024);
-            constexpr uint32_t id1 = idesc_tf32(128, 64, false, false);
+            const uint64_t by = sw128_desc(sbase + OFF_Y, 16, 1024);
+            constexpr uint32_t id1 = idesc_tf32(128, 160, false, false);
 #pragma unroll
             for (int kk = 0; kk < DK / 8; ++kk)
-                mma_tf32_ts(tmem + TM_D1, tmem + TM_A1 + 8 * kk, bkm + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4),
-                            id1, kk > 0);
-            mma_commit(bar_mma);
+                mma_tf32_ts(tmem + TM_D1, tmem + TM_X + 8 * kk, by + (((kk >> 2) * 160 * 128 + (kk & 3) * 32) >> 4), id1,
+                            kk > 0);
+            mma_commit(bar_m1);
         }
-        failed = !mbar_wait(bar_mma, 0, kWaitPolls);  // bar_mma completes twice per task: parities 0, 1
+        failed = !mbar_wait(bar_m1, par, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        {   // rows 0..63 -> A (beta-scaled, strictly lower, fp32); rows 64..127 -> P (lower, tf32 operand)
-            float x[16];
-            tmem_ld16(tq + TM_D1 + 16 * qr, x);
-            const int col0 = 16 * qr;
-            if (c < C) {
-                const float b = s_beta[c];
-                float* arow = reinterpret_cast<float*>(sm + OFF_A) + c * TP + col0;
+        {   // lane rows 0..63 -> A (beta-scaled, strictly lower, fp32); 64..127 -> P (lower with the
+            // diagonal).  Lanes 0-15 of the warp are rows of block R0, lanes 16-31 of block R0 + 1; the
+            // warp reads its blocks' columns in 16-column pieces, the four warps of a quadrant in turn.
+            const bool isq = c >= 64;
+            const int row = c & 63, Rl = row >> 4;
+            const int R0 = 2 * (q4 & 1), n0 = R0 + 1, ntot = 2 * R0 + 3;
+            const float b = s_beta[row];
+            for (int ch = qr; ch < ntot; ch += 4) {
+                const int R = ch < n0 ? R0 : R0 + 1;
+                const int j16 = ch < n0 ? ch : ch - n0;
+                float x[16];
+                tmem_ld16(tq + TM_D1 + y_row(R) + 16 * j16, x);
+                if (Rl != R) continue;
+                const int i0 = 16 * j16;
+                if (!isq) {
+                    float* arow = reinterpret_cast<float*>(sm + OFF_A) + row * TP + i0;
 #pragma unroll
-                for (int k4 = 0; k4 < 16; k4 += 4) {
-                    float a[4];
+                    for (int k4 = 0; k4 < 16; k4 += 4) {
+                        float a[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) a[u] = (col0 + k4 + u) < c ? b * x[k4 + u] : 0.f;
-                    *reinterpret_cast<float4*>(arow + k4) = make_float4(a[0], a[1], a[2], a[3]);
+                        for (int u = 0; u < 4; ++u) a[u] = (i0 + k4 + u) < row ? b * x[k4 + u] : 0.f;
+                        *reinterpret_cast<float4*>(arow + k4) = make_float4(a[0], a[1], a[2], a[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int k4 = 0; k4 < 16; k4 += 4) {
+                        float p[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) p[u] = (i0 + k4 + u) <= row ? x[k4 + u] : 0.f;
+                        if (!any_strong)
+                            *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + row, i0 + k4, 192)) =
+                                make_float4(to_tf32(p[0]), to_tf32(p[1]), to_tf32(p[2]), to_tf32(p[3]));
+                        else
+                            *reinterpret_cast<float4*>(sm + OFF_PF + pf_off(row, i0 + k4)) = make_float4(p[0], p[1], p[2], p[3]);
+                    }
                 }
-            } else {
-                const int t = c - C;
+            }
+            if (isq && qr > Rl) {  // P above the row's block: zeros
 #pragma unroll
                 for (int k4 = 0; k4 < 16; k4 += 4) {
-                    float p[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) p[u] = (col0 + k4 + u) <= t ? to_tf32(x[k4 + u]) : 0.f;
-                    *reinterpret_cast<float4*>(sm + OFF_P + sw128_off(t, col0 + k4, 64)) = make_float4(p[0], p[1], p[2], p[3]);
+                    if (!any_strong)
+                        *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + row, 16 * qr + k4, 192)) =
+                            make_float4(0.f, 0.f, 0.f, 0.f);
+                    else
+                        *reinterpret_cast<float4*>(sm + OFF_PF + pf_off(row, 16 * qr + k4)) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
         }
+        if (any_strong) {
+            // exact terms of the strong-decay channels inside each diagonal block: thread (row, qr) adds,
+            // over the strong channels 32 qr .. 32 qr + 31 of its row's block, x_rc k_ic e^{g_rc - g_ic}
+            __syncthreads();
+            const bool isq = c >= 64;
+            const int row = c & 63, Rl = row >> 4, b0 = 16 * Rl;
+            if (row < len) {
+                float acc[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+                for (uint32_t m = s_strong[Rl * 4 + qr]; m; m &= m - 1) {
+                    const int ch = 32 * qr + __ffs(m) - 1;
+                    const float xr = __bfloat162float((isq ? sq : sk)[bf16_sw_off(row, ch) >> 1]) *
+                                     (PRO ? s_rn[isq ? 64 + row : row] : 1.f);
+                    const float gr = gf_at(row, ch);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int i = b0 + j;
+                        if (i < row || (isq && i == row)) {
+                            const float ki = __bfloat162float(sk[bf16_sw_off(i, ch) >> 1]) * (PRO ? s_rn[i] : 1.f);
+                            acc[j] += xr * ki * __expf(gr - gf_at(i, ch));
+                        }
+                    }
+                }
+                if (!isq) {
+                    const float bb = s_beta[row];
+                    float* arow = reinterpret_cast<float*>(sm + OFF_A) + row * TP + b0;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (b0 + j < row) atomicAdd(arow + j, bb * acc[j]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (b0 + j <= row) atomicAdd(reinterpret_cast<float*>(sm + OFF_PF + pf_off(row, b0 + j)), acc[j]);
+                }
+            }
+            __syncthreads();
+            {   // P -> its tf32 operand rows of [Kt; P]
+                const int t = tid >> 3, i8 = (tid & 7) * 8;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float4 p = *reinterpret_cast<const float4*>(sm + OFF_PF + pf_off(t, i8 + 4 * h));
+                    *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + t, i8 + 4 * h, 192)) =
+                        make_float4(to_tf32(p.x), to_tf32(p.y), to_tf32(p.z), to_tf32(p.w));
+                }
+            }
+        }
+        // the staging buffers are read: the next task's tiles may come in while this one finishes
+        const Task tn = slots[nxt];
+        if (tid == 0 && tn.id >= 0) {
+            mbar_arrive_expect_tx(bar_tma, kStageBytes);
+            ++loads_issued;
+        }
         __syncthreads();
+        if (lane == 0 && warp < kLoads && tn.id >= 0) load_box(tn, warp);
+        load_beta(tn, par ^ 1u);
 
         // ---- T = (I + A)^{-1}, then its tf32 operand tile
         unit_lower_inverse(reinterpret_cast<const float*>(sm + OFF_A), reinterpret_cast<float*>(sm + OFF_T32), xs);
@@ -540,76 +773,64 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_before_sync();
         __syncthreads();
 
-        // ---- MMA 2: [W | U] = T [beta K e^G | beta V]   (M=64, N=256, K=64)
+        // ---- MMA 2: W^T = (beta K e^G)^T T^T, U^T = (beta V)^T T^T   (M=128, N=64, K=64; A in tensor memory)
         if (tid == 0) {
             tc_fence_after_sync();
-            const uint64_t at = sw128_desc(sbase + OFF_TIMG, 16, 1024);
-            const uint64_t b8 = sw128_desc(sbase + OFF_B8, 16, 1024);
-            constexpr uint32_t id8 = idesc_tf32(64, 256, false, false);
+            const uint64_t bt = sw128_desc(sbase + OFF_TIMG, 16, 1024);
+            constexpr uint32_t id2 = idesc_tf32(128, 64, false, false);
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)
-                mma_tf32(tmem + TM_D8, at + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4),
-                         b8 + (((kk >> 2) * 32768 + (kk & 3) * 32) >> 4), id8, kk > 0);
-            mma_commit(bar_mma);
+            for (int kk = 0; kk < C / 8; ++kk) {
+                const uint64_t b = bt + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
+                mma_tf32_ts(tmem + TM_WT, tmem + TM_BK + 8 * kk, b, id2, kk > 0);
+                mma_tf32_ts(tmem + TM_UT, tmem + TM_BV + 8 * kk, b, id2, kk > 0);
+            }
+            mma_commit(bar_m2);
         }
         if (tid == kWalker) slots[aft] = walker.next();  // while MMA 2 runs: the task after the next
-        failed = !mbar_wait(bar_mma, 1, kWaitPolls);
+        failed = !mbar_wait(bar_m2, par, kWaitPolls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        {   // [W | U] (M=64 layout: row s = 16 q4 + lane % 16), columns 64 qr + 32 (lane / 16) .. +31
-            // -> MN-major over B8
+        {   // -W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..)
             float x[32];
-            tmem_ld32_x2<32>(tq + TM_D8 + 64 * qr, x);
-            const int s = 16 * q4 + (lane & 15);
+            const bool isw = qr < 2;
+            tmem_ld32(tq + (isw ? TM_WT : TM_UT) + 32 * (qr & 1), x);
+            const float sgn = isw ? -1.f : 1.f;
+            unsigned char* tile = sm + (isw ? OFF_WT : OFF_UT);
 #pragma unroll
-            for (int e8 = 0; e8 < 4; ++e8) {
-                const int n0 = 64 * qr + 32 * (lane >> 4) + 8 * e8;
-                float4* d = reinterpret_cast<float4*>(sm + OFF_B8 + sw32b_off(s, n0, 64));
-                d[0] = make_float4(to_tf32(x[8 * e8]), to_tf32(x[8 * e8 + 1]), to_tf32(x[8 * e8 + 2]),
-                                   to_tf32(x[8 * e8 + 3]));
-                d[1] = make_float4(to_tf32(x[8 * e8 + 4]), to_tf32(x[8 * e8 + 5]), to_tf32(x[8 * e8 + 6]),
-                                   to_tf32(x[8 * e8 + 7]));
-            }
+            for (int e4 = 0; e4 < 32; e4 += 4)
+                *reinterpret_cast<float4*>(tile + sw128_off(c, 32 * (qr & 1) + e4, 128)) =
+                    make_float4(to_tf32(sgn * x[e4]), to_tf32(sgn * x[e4 + 1]), to_tf32(sgn * x[e4 + 2]), to_tf32(sgn * x[e4 + 3]));
         }
         fence_async_smem();
         tc_fence_before_sync();
         __syncthreads();
 
-        // ---- MMA 3: P W (M=64, N=128);  MMA 4: Kt^T W (M=128, N=128);  MMA 5: B^T = U^T Kt (M=128, N=128);
-        //      MMA 6: Uo^T = U^T P^T (M=128, N=64).  K = 64 (tokens s) throughout; W and U from the MN-major
-        //      [W | U] tile (U^T as an MN-major A operand), Kt and P as K-major A or B operands.
+        // ---- MMA 3: [-W^T Kt | -W^T P^T] (= Mt^T - Diag(e^{g_C}) | Qh^T - (Q e^G)^T);  MMA 4: [U^T Kt | U^T P^T]
+        //      (= B^T | Uo^T).  M=128, N=192 ([Kt; P] rows), K=64 (tokens s); A and B in shared memory.
         if (tid == 0) {
             tc_fence_after_sync();
-            const uint64_t bw = sw128b32_desc(sbase + OFF_B8, 64 * 128, 512);
-            const uint64_t au = sw128b32_desc(sbase + OFF_B8 + 4 * 64 * 128, 64 * 128, 512);
-            const uint64_t dkt = sw128_desc(sbase + OFF_KT, 16, 1024);
-            const uint64_t dp = sw128_desc(sbase + OFF_P, 16, 1024);
-            constexpr uint32_t id_pw = idesc_tf32(64, 128, false, true);
-            constexpr uint32_t id_kw = idesc_tf32(128, 128, false, true);
-            constexpr uint32_t id_bt = idesc_tf32(128, 128, true, false);
-            constexpr uint32_t id_ut = idesc_tf32(128, 64, true, false);
-            // B^T and Uo^T first: their read-out and stores to the record overlap MMAs 3 and 4
+            const uint64_t aw = sw128_desc(sbase + OFF_WT, 16, 1024);
+            const uint64_t au = sw128_desc(sbase + OFF_UT, 16, 1024);
+            const uint64_t bkp = sw128_desc(sbase + OFF_KP, 16, 1024);
+            constexpr uint32_t id3 = idesc_tf32(128, 192, false, false);
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk) {
-                const uint64_t mn = static_cast<uint64_t>(kk) * 64;
-                mma_tf32(tmem + TM_BT, au + mn, dkt + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), id_bt, kk > 0);
-                mma_tf32(tmem + TM_UT, au + mn, dp + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_ut, kk > 0);
-            }
-            mma_commit(bar_bu);
+            for (int kk = 0; kk < C / 8; ++kk)
+                mma_tf32(tmem + TM_DU, au + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                         bkp + (((kk >> 2) * 24576 + (kk & 3) * 32) >> 4), id3, kk > 0);
+            mma_commit(bar_m4);
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk) {
-                const uint64_t mn = static_cast<uint64_t>(kk) * 64;
-                mma_tf32(tmem + TM_PW, dp + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), bw + mn, id_pw, kk > 0);
-                mma_tf32(tmem + TM_KW, dkt + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), bw + mn, id_kw, kk > 0);
-            }
-            mma_commit(bar_rest);
+            for (int kk = 0; kk < C / 8; ++kk)
+                mma_tf32(tmem + TM_DW, aw + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                         bkp + (((kk >> 2) * 24576 + (kk & 3) * 32) >> 4), id3, kk > 0);
+            mma_commit(bar_m3);
         }
-        failed = !mbar_wait(bar_bu, it & 1, kWaitPolls);
-        if (__syncthreads_or(failed)) { failed = true; break; }
+        // a timed-out wait here is acted on at the end of the task (the read-outs below then only
+        // write garbage into this task's own record)
+        bool late = !mbar_wait(bar_m4, par, kWaitPolls);
         tc_fence_after_sync();
         {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record
             float x[32];
-            tmem_ld32(tq + TM_BT + 32 * qr, x);
+            tmem_ld32(tq + TM_DU + 32 * qr, x);
             float m = 0.f;
 #pragma unroll
             for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(x[e]));
@@ -630,69 +851,39 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             reinterpret_cast<signed char*>(rec + wy::REC_BEXP)[qr * 128 + c] = static_cast<signed char>(ex);
             float y[16];
-            tmem_ld16(tq + TM_UT + 16 * qr, y);
+            tmem_ld16(tq + TM_DU + 128 + 16 * qr, y);
             float4* gu = reinterpret_cast<float4*>(rec + wy::REC_UO);
 #pragma unroll
             for (int s4 = 0; s4 < 4; ++s4)
                 gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4], y[4 * s4 + 1], y[4 * s4 + 2], y[4 * s4 + 3]);
         }
-        failed = !mbar_wait(bar_rest, it & 1, kWaitPolls);
-        if (__syncthreads_or(failed)) { failed = true; break; }
+        late |= !mbar_wait(bar_m3, par, kWaitPolls);
         tc_fence_after_sync();
-        {   // Qh = Q e^G - P W (row t = 16 q4 + lane % 16, channels 32 qr + 16 (lane / 16) ..) -> staging,
-            // K-major rows t
-            const int t = 16 * q4 + (lane & 15), hc = lane >> 4;
-            const bool live = t < len;
-            const float rq = PRO ? s_rn[64 + t] : 1.f;
-            float x[16];
-            tmem_ld16_x2<16>(tq + TM_PW + 32 * qr, x);
-            unsigned char* row = sm + STG_Q + qr * 8192 + t * 128;  // K-block qr, row t
-#pragma unroll
-            for (int e8 = 0; e8 < 2; ++e8) {
-                const int cc = 32 * qr + 16 * hc + 8 * e8;
-                float qv[8];
-                unpack8(*reinterpret_cast<const uint4*>(sm + OFF_SQ + bf16_sw_off(t, cc)), qv);
-                const float4 e0 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc, 64));
-                const float4 e1 = *reinterpret_cast<const float4*>(sm + OFF_G + sw128_off(t, cc + 4, 64));
-                const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-                float qh[8];
-#pragma unroll
-                for (int w = 0; w < 8; ++w)
-                    qh[w] = to_tf32((live ? qv[w] * rq * ev[w] * x_egm[cc + w] : 0.f) - x[8 * e8 + w]);
-                const int ch = 4 * hc + 2 * e8;  // 16-byte chunk of the row within the K-block
-                *reinterpret_cast<float4*>(row + ((ch ^ (t & 7)) << 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
-                *reinterpret_cast<float4*>(row + (((ch + 1) ^ (t & 7)) << 4)) = make_float4(qh[4], qh[5], qh[6], qh[7]);
-            }
-        }
-        const Task tn = slots[nxt];
-        if (tid == 0 && tn.id >= 0) {
-            mbar_arrive_expect_tx(bar_tma, kStageBytes);
-            ++loads_issued;
-        }
-        __syncthreads();  // q and E are read: the next task's tiles may come into the staging buffers
-        if (lane == 0 && warp < kLoads && tn.id >= 0) load_box(tn, warp);
-        load_beta(tn, (it + 1) & 1);
-        {   // Mt = Diag(e^{g_C}) - Kt^T W (row i = c, columns j = 32 qr ..) -> staging, K-major rows i
+        {   // Mt (lane j = c, rows i = 32 qr ..) and Qh (lane j, tokens t = 16 qr ..) into their record tiles
+            // in shared memory (for each i or t the warp's 32 lanes write one 128-byte row), then two bulk
+            // copies.  The [Kt; P] and W^T, U^T tiles under them are dead: MMAs 3 and 4 are complete.
             float x[32];
-            tmem_ld32(tq + TM_KW + 32 * qr, x);
-            const float gam = x_gam[c];
-            unsigned char* row = sm + STG_M + qr * 16384 + c * 128;  // K-block qr, row i
+            tmem_ld32(tq + TM_DW + 32 * qr, x);
+            const float gam = s_gam[c];
+            unsigned char* stm = sm + OFF_STM + q4 * 16384 + ((lane & 3) << 2);
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                float m[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) m[u] = to_tf32((c == 32 * qr + 4 * e4 + u ? gam : 0.f) - x[4 * e4 + u]);
-                *reinterpret_cast<float4*>(row + ((e4 ^ (c & 7)) << 4)) = make_float4(m[0], m[1], m[2], m[3]);
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * qr + e;  // row i of K-block q4 of Mt; its 16-byte chunks permuted by i % 8 = e % 8
+                *reinterpret_cast<float*>(stm + i * 128 + (((lane >> 2) ^ (e & 7)) << 4)) = to_tf32(x[e] + (i == c ? gam : 0.f));
             }
+            float y[16], sd[16];
+            tmem_ld16(tq + TM_DW + 128 + 16 * qr, y);
+            tmem_ld16(tq + TM_QG + 16 * qr, sd);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                *reinterpret_cast<float*>(sm + OFF_STQ + sw128_off(16 * qr + e, c, 64)) = to_tf32(y[e] + sd[e]);
         }
         fence_async_smem();
         tc_fence_before_sync();
-        __syncthreads();
+        if (__syncthreads_or(late)) { failed = true; break; }
         if (tid == 0) {
-#pragma unroll
-            for (int b = 0; b < 4; ++b) bulk_store(rec + wy::REC_M + b * 16384, sm + STG_M + b * 16384, 16384);
-            bulk_store(rec + wy::REC_Q, sm + STG_Q, 16384);
-            bulk_store(rec + wy::REC_Q + 16384, sm + STG_Q + 16384, 16384);
+            bulk_store(rec + wy::REC_M, sm + OFF_STM, 65536);
+            bulk_store(rec + wy::REC_Q, sm + OFF_STQ, 32768);
             bulk_commit();
         }
     }
@@ -702,7 +893,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (loads_issued > 0) mbar_wait(bar_tma, (loads_issued - 1) & 1, kWaitPolls);
         raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
     }
-    if (tid == 0) bulk_wait_read();  // the bulk stores read shared memory until they complete
+    if (tid == 0) bulk_wait_read();  // the bulk copies read shared memory until they complete
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {

@@ -65,11 +65,8 @@ inline bool chunk_tc_path(int64_t T_total, kda_dtype dtype_qkv, int dk, int dv) 
 // Each launcher returns cudaSuccess or the launch error.
 cudaError_t launch_decode(const DecodeArgs& a);
 cudaError_t launch_chunk_simt(const ChunkArgs& a);
-// bf16, dk = dv = 128: the tensor-core paths.  With a workspace of chunk_wy_workspace_size bytes the
-// chunk-local kernel (launch_chunk_prep) writes every chunk's record and the scan (launch_chunk_scan)
-// walks them; without one, launch_chunk_tc does both in one kernel per (sequence, head, dv slice).
-bool chunk_tc_supported(const ChunkArgs& a);
-cudaError_t launch_chunk_tc(const ChunkArgs& a);
+// bf16, dk = dv = 128 with a workspace of chunk_wy_workspace_size bytes: the chunk-local kernel
+// (launch_chunk_prep) writes every chunk's record, then the scan (launch_chunk_scan) walks them.
 size_t chunk_wy_workspace_size(int64_t T_total, int N, int H, int dk, int dv);
 // The scan's part of that workspace, after the records: two fp32 [N, H, dk, dv] state arrays.
 size_t chunk_scan_state_bytes(int N, int H);

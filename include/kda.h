@@ -21,9 +21,9 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Calls are
  *     asynchronous on that stream: a returned KDA_OK means "validated and launched".
  *   - Arguments are validated on the host before any launch; an invalid argument returns a status
- *     and launches nothing.  Problems only the device can see (the contents of cu_seqlens, a decay
- *     range the tensor-core path cannot represent) set sticky flags that kda_get_device_status
- *     reads.  Nothing traps or asserts on the device.
+ *     and launches nothing.  Problems only the device can see (the contents of cu_seqlens, a bounded
+ *     wait that gave up) set sticky flags that kda_get_device_status reads.  Nothing traps or
+ *     asserts on the device.
  *   - dtypes: q/k/v share `dtype_qkv`; log_alpha/beta share `dtype_gate`; o has `dtype_o`.
  *     The recurrent state is always fp32.
  */
@@ -57,10 +57,8 @@ typedef enum { KDA_BF16 = 0, KDA_FP32 = 1 } kda_dtype;
 /* Sticky device flags returned by kda_get_device_status (bitwise OR). */
 #define KDA_DEVFLAG_CU_SEQLENS 0x1u   /* cu_seqlens[0] != 0, decreasing, or cu_seqlens[N] != T_total;
                                          the offending sequences were skipped */
-#define KDA_DEVFLAG_DECAY_RANGE 0x2u  /* within some 64-token chunk the cumulative log-decay moved by
-                                         more than 80 (nats) between the chunk's middle row and its
-                                         first or last row; the bf16 tensor-core path's outputs for
-                                         that chunk are not reliable (the fp32 path is exact there) */
+#define KDA_DEVFLAG_DECAY_RANGE 0x2u  /* reserved (bit kept for ABI stability): no path raises it, since
+                                         every path is exact for every decay in (0, 1) */
 #define KDA_DEVFLAG_TIMEOUT 0x4u      /* a bounded inter-CTA wait gave up */
 
 /*
@@ -95,11 +93,14 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int64_t T_total, int N, int H, int d
  *               garbage on exit.  A non-NULL workspace smaller than the size returns
  *               KDA_ERR_INVALID_ARG.
  *
- * Path: dtype_qkv == KDA_FP32 runs the fp32 CUDA-core path (every product in fp32; no workspace
- * used).  KDA_BF16 with dk = dv = 128 runs on the tensor cores (tf32 products, fp32 accumulation and
- * fp32 state): with the workspace, a chunk-local kernel over all chunks at once followed by a scan
- * over each sequence's chunks (about 2.5 KB of workspace per token and head); without it, one kernel
- * per (sequence, head, 32-column slice of dv) that does both, slower.
+ * Path: KDA_BF16 with dk = dv = 128 and a workspace runs on the tensor cores (tf32 products, fp32
+ * accumulation and fp32 state): a chunk-local kernel over all chunks at once followed by a scan over
+ * each sequence's chunks (about 2.5 KB of workspace per token and head).  Every other call -- fp32
+ * q/k/v, dk or dv = 64, or no workspace -- runs the CUDA-core path (every product in fp32, no
+ * workspace used), which is exact at fp32 tolerances but several times slower on long sequences.
+ * Both paths are exact up to rounding for every decay: within a chunk the decay factors are split
+ * at 16-row block boundaries so that none exceeds e^40, and strongly decaying channels take exact
+ * per-element factors.
  */
 KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          const void* log_alpha, const void* beta,

@@ -60,8 +60,8 @@ def test_ragged_varlen(dtype, dk, dv):
 
 
 @pytest.mark.parametrize("case", ["ragged", "bf16_gates", "b2_h4_t2048"])
-def test_workspace_free_kernel(case):
-    """Without a workspace the bf16 dk = dv = 128 path runs the single fused kernel."""
+def test_workspace_free_path(case):
+    """Without a workspace the bf16 dk = dv = 128 call runs the CUDA-core path (fp32 products)."""
     if case == "ragged":
         inp = gen.make_prefill([1, 63, 64, 65, 130, 0, 200, 7], 3, 128, 128, init_state=True, seed=21, device=DEV)
     elif case == "bf16_gates":
@@ -284,24 +284,34 @@ def _with_gates(inp, log_alpha_value=None, beta_value=None):
 @pytest.mark.parametrize("case", ["no_decay", "beta_zero", "beta_one", "strong_decay_in_range"])
 def test_degenerate_gates(dtype, d, case):
     """alpha = 1 (log_alpha = 0: the plain delta rule), beta = 0 (pure decay), beta = 1 (full
-    overwrite), and a decay whose cumulative log over a chunk reaches 76.8 nats on each side of the
-    anchor row -- inside the tensor-core path's 80-nat range -- all against the oracle."""
+    overwrite), and a steady decay of 2.4 nats per token (a 16-row block spans 36 nats), all against
+    the oracle."""
     inp = gen.make_prefill([200, 64, 129], 2, d, d, dtype=dtype, init_state=True, seed=27, device=DEV)
     la = {"no_decay": 0.0, "strong_decay_in_range": -2.4}.get(case)
     b = {"beta_zero": 0.0, "beta_one": 1.0}.get(case)
     _check_full(_with_gates(inp, la, b), dtype)
 
 
-def test_decay_beyond_the_anchor_range():
-    """log_alpha = -5 per token: the cumulative decay spans 160 nats on either side of a chunk's anchor.
-    The tf32 tensor-core path flags the chunks (KDA_DEVFLAG_DECAY_RANGE) instead of returning silently;
-    the fp32 path evaluates those chunks exactly and matches the oracle."""
-    inp = _with_gates(gen.make_prefill([300], 2, 128, 128, init_state=True, seed=28, device=DEV), -5.0)
-    kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, inp.cu_seqlens,
-                      dtype_o=torch.float32)
-    st, flags = kda.kda_get_device_status()
-    assert st == kda.KDA_ERR_DEVICE_CHECK and flags & kda.KDA_DEVFLAG_DECAY_RANGE
-    assert kda.kda_get_device_status() == (kda.KDA_OK, 0)
-    inp32 = _with_gates(gen.make_prefill([300], 2, 128, 128, dtype=torch.float32, init_state=True, seed=28,
-                                         device=DEV), -5.0)
-    _check_full(inp32, torch.float32)
+@pytest.mark.parametrize("use_workspace", [True, False])
+@pytest.mark.parametrize("log_alpha", [-5.0, -20.0, -1e4])
+def test_strong_decay_matches_oracle(log_alpha, use_workspace):
+    """A decay of 5, 20 or 10^4 nats per token in every channel (alpha = 6.7e-3, 2e-9, ~0: the last is
+    the reset the recurrence allows as alpha -> 0).  At 5 nats a 16-row block spans 75 nats and stays
+    in the tensor-core products; at 20 and 10^4 every channel takes the exact per-element terms inside
+    the diagonal blocks.  Both prefill paths match the oracle and raise no flag."""
+    inp = _with_gates(gen.make_prefill([300, 64, 129], 2, 128, 128, init_state=True, seed=28, device=DEV), log_alpha)
+    _check_full(inp, torch.bfloat16, use_workspace=use_workspace)
+
+
+@pytest.mark.parametrize("use_workspace", [True, False])
+def test_mixed_strong_and_weak_channels_match_oracle(use_workspace):
+    """Per-token decays drawn from the workload's distribution, with a third of the channels (chosen at
+    random per head) decaying at 20 nats per token and a few tokens of the others at 60: blocks mix
+    channels in the tensor-core products with channels on the exact per-element path."""
+    inp = gen.make_prefill([300, 64, 129, 1], 3, 128, 128, init_state=True, seed=29, device=DEV)
+    g = torch.Generator(device="cpu").manual_seed(29)
+    strong = (torch.rand((1, inp.H, inp.dk), generator=g) < 1 / 3).to(DEV)
+    spikes = (torch.rand((inp.T_total, inp.H, 1), generator=g) < 0.02).to(DEV)
+    la = torch.where(strong, torch.full_like(inp.log_alpha, -20.0), inp.log_alpha)
+    inp.log_alpha = torch.where(spikes & ~strong, torch.full_like(la, -60.0), la)
+    _check_full(inp, torch.bfloat16, use_workspace=use_workspace)
