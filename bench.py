@@ -11,6 +11,10 @@ One step = one pass of the whole hot path over one batch of synthetic input:
 `value` is prefill tokens/s over all ranks (B*T*N / max-over-ranks prefill time); the decode leg is
 reported in "decode" (state GB/s, tokens/s).  Inputs stay resident in HBM during the timed region;
 every input is larger than the 126 MB L2, so no flush is needed between steps.
+After the timed steps two more legs run (skipped with --no-extra): "varlen", the packed varlen prefill
+(16 sequences, about 670k tokens, 32 heads -- the largest single-GPU prefill), and "decode_stream",
+the decode workload as specified (1024 successive steps, each with its own inputs, back to back), with
+its own end-to-end figure (per-step inputs copied in from pinned host memory, o copied back).
 Each rank runs its own independent copy of the workload (no data-path collective; weak scaling).
 
 `--impl reference` times the fp64 CPU oracle instead (the reference arm), on a bounded sample of
@@ -33,6 +37,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 PREFILL = "prefill_b1_h32_t32768"
+VARLEN = "varlen_n16_h32"
 DECODE = "decode_b256_h32"
 # Algorithmic bytes per token-head of a fully fused prefill: q, k, v bf16 (3 * 128 * 2), log_alpha fp32
 # (128 * 4), beta fp32 (4), o bf16 (128 * 2).  Useful flops per token-head: 6 dk dv + C (3 dk + 2 dv).
@@ -58,6 +63,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the varlen prefill leg and the 1024-step decode stream")
     p.add_argument("--only", choices=["prefill", "decode"], default=None,
                    help="profiling aid: run only one leg (with --no-e2e --no-cpu-baseline)")
     p.add_argument("--prefill-tokens", type=int, default=None,
@@ -188,25 +195,20 @@ def sources_digest(paths):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(summary_name: str, sources):
-    """dram bytes per launch from a committed ncu summary, or None if absent or if the kernel source
-    changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", summary_name)
+def profiled_traffic(key: str, sources):
+    """DRAM bytes per call from profiles/traffic.json (written from an ncu capture; see the summaries
+    beside it), or None if absent or if a kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            text = f.read()
-    except OSError:
+            entry = json.load(f)[key]
+    except (OSError, KeyError, ValueError):
         return None
-    fields = {}
-    for line in text.splitlines():
-        if ":" in line and line.lstrip().startswith("- "):
-            key, val = line.lstrip()[2:].split(":", 1)
-            fields[key.strip()] = val.strip().strip("`")
-    if fields.get("kernel_source_digest") != sources_digest(sources):
+    if entry.get("kernel_source_digest") != sources_digest(sources):
         return None
     try:
-        return float(fields["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return float(entry["dram_bytes_per_call"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -285,6 +287,122 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------------------------ our arm
+
+def time_calls(fn, stream, n):
+    """Median CUDA-event time (ms) of n calls of fn on `stream`, each bracketed by its own events."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+
+def varlen_leg(gen, kda, device, stream, rank, dist, world, hbm_peak):
+    """The varlen workload (16 packed sequences, lengths U[1024, 65536], 32 heads): the largest
+    single-GPU prefill.  3 timed calls after one warm-up; tokens/s over all ranks and its roofline."""
+    w = gen.WORKLOADS[VARLEN]
+    inp = gen.make_workload(VARLEN, seed=rank, device=device)
+    T, H, N = inp.T_total, inp.H, inp.N
+    o = torch.empty((T, H, inp.dv), dtype=torch.bfloat16, device=device)
+    sf = torch.empty((N, H, inp.dk, inp.dv), dtype=torch.float32, device=device)
+    ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(T, N, H, inp.dk, inp.dv), 1), dtype=torch.uint8, device=device)
+    call = lambda: kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state, inp.cu_seqlens,
+                                     o=o, final_state=sf, workspace=ws, stream=stream)
+    call()
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    ms = max_over_ranks(time_calls(call, stream, 3), dist, device)
+    st, flags = kda.kda_get_device_status(stream)
+    if st != kda.KDA_OK:
+        raise SystemExit(f"device status after the varlen leg: {st} flags {flags:#x}")
+    # algorithmic bytes: every input and o once, plus the initial and final states
+    nbytes = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * N * H * inp.dk * inp.dv * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out = {"workload": f"{VARLEN}: N={N} sequences (lengths U[{w['len_lo']}, {w['len_hi']}], {T} tokens), H={H}, "
+                       f"dk=dv=128, chunk 64, bf16 q/k/v, fp32 gates and states, bf16 o",
+           "tokens": T, "ms_per_call": ms, "value": world * T * 1000.0 / ms, "unit": "tokens/s",
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                        "algorithmic_bytes_per_launch": nbytes},
+           "launches_per_call": PREFILL_KERNELS_PER_CALL}
+    del inp, o, sf, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def decode_stream_leg(gen, kda, device, stream, rank, dist, world, hbm_peak, e2e_steps):
+    """The decode workload as specified: 1024 successive single-token steps over 256 x 32 fp32 states,
+    each with its own inputs (all resident in HBM beforehand), launched back to back; per-step CUDA-event
+    times, median reported.  Then the same stream end to end for `e2e_steps` steps: each step's inputs
+    copied in from pinned host memory and its o copied back, inside the timed region."""
+    w = gen.WORKLOADS[DECODE]
+    B, H, dk, dv, steps = w["B"], w["H"], w["dk"], w["dv"], w["steps"]
+    xs = [gen.make_decode_step(i, B, H, dk, dv, seed=rank, device=device) for i in range(steps)]
+    state0 = gen.make_decode_state(B, H, dk, dv, seed=rank, device=device)
+    state = state0.clone()
+    o = torch.empty((B, H, dv), dtype=torch.bfloat16, device=device)
+    step = lambda x, st: kda.kda_decode_step(x.q, x.k, x.v, x.log_alpha, x.beta, st, o=o, stream=stream)
+    for i in range(3):  # warm-up on a copy of the state, then the stream from the initial state
+        step(xs[i], state)
+    state.copy_(state0)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        step(xs[i], state)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    per_step = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(steps))
+    med = max_over_ranks(statistics.median(per_step), dist, device)
+    total = max_over_ranks(ev[0].elapsed_time(ev[steps]), dist, device)
+    st, flags = kda.kda_get_device_status(stream)
+    if st != kda.KDA_OK:
+        raise SystemExit(f"device status after the decode stream: {st} flags {flags:#x}")
+    nbytes = B * H * DECODE_BYTES_PER_HEAD
+    gbs = nbytes / (med * 1e-3) / 1e9
+    out = {"workload": f"{DECODE}: B={B}, H={H}, dk=dv=128, fp32 states, {steps} successive steps, per-step bf16 "
+                       f"q/k/v and fp32 gates, bf16 o",
+           "steps": steps, "us_per_step_median": 1000.0 * med, "us_per_step_mean": 1000.0 * total / steps,
+           "us_per_step_p90": 1000.0 * per_step[int(0.9 * (steps - 1))],
+           "tokens_per_s": world * B * 1000.0 / med, "state_gbs": world * nbytes / (med * 1e-3) / 1e9,
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                        "frac_of_8tbs": gbs / 8000.0, "algorithmic_bytes_per_launch": nbytes},
+           "launches": steps}
+    if e2e_steps > 0:
+        names = ("q", "k", "v", "log_alpha", "beta")
+        host = [{n: getattr(xs[i], n).cpu().pin_memory() for n in names} for i in range(e2e_steps)]
+        dev_in = {n: torch.empty_like(getattr(xs[0], n)) for n in names}
+        o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host[0].values())
+        d2h = o_host.numel() * o_host.element_size()
+        state.copy_(state0)
+
+        def e2e_step(i):
+            for n in names:
+                dev_in[n].copy_(host[i][n], non_blocking=True)
+            kda.kda_decode_step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["log_alpha"], dev_in["beta"], state,
+                                o=o, stream=stream)
+            o_host.copy_(o, non_blocking=True)
+        e2e_step(0)
+        state.copy_(state0)
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, device)
+        out["e2e"] = {"value": world * B * 1000.0 / ms, "unit": "tokens/s", "us_per_step": 1000.0 * ms,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+        del host, dev_in, o_host
+    del xs, state, state0
+    torch.cuda.empty_cache()
+    return out
+
 
 def run_ours(args):
     from gated_delta_rule_127_b200 import inputs as gen
@@ -402,14 +520,19 @@ def run_ours(args):
         raise SystemExit(f"device status after timing: {st} flags {flags:#x}")
 
     hbm_peak, tf_peak, peak_src = measured_peaks()
+    varlen = dec_stream = None
+    if not args.no_extra and args.only is None and args.prefill_tokens is None:
+        varlen = varlen_leg(gen, kda, device, stream, rank, dist, world, hbm_peak)
+        dec_stream = decode_stream_leg(gen, kda, device, stream, rank, dist, world, hbm_peak,
+                                       0 if args.no_e2e else 64)
     token_heads = T * H
     prefill_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD
     prefill_flops = token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD
     achieved_gbs = prefill_bytes / (prefill_local * 1e-3) / 1e9
-    traffic = profiled_traffic("kda_chunk_fwd_prefill_b1_h32_t32768.md", PREFILL_KERNEL_SOURCES)
+    traffic = profiled_traffic("kda_chunk_fwd prefill_b1_h32_t32768", PREFILL_KERNEL_SOURCES)
     dec_bytes = Bd * Hd * DECODE_BYTES_PER_HEAD
     dec_gbs = dec_bytes / (decode_local * 1e-3) / 1e9
-    dec_traffic = profiled_traffic("kda_decode_step_decode_b256_h32.md", DECODE_KERNEL_SOURCES)
+    dec_traffic = profiled_traffic("kda_decode_step decode_b256_h32", DECODE_KERNEL_SOURCES)
 
     line = None
     if rank == 0:
@@ -442,7 +565,12 @@ def run_ours(args):
                          "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": prefill_bytes,
                          "tensor_tflops": prefill_flops / (prefill_local * 1e-3) / 1e12,
-                         "tensor_frac": prefill_flops / (prefill_local * 1e-3) / 1e12 / tf_peak},
+                         "tensor_frac": prefill_flops / (prefill_local * 1e-3) / 1e12 / tf_peak,
+                         "tensor_frac_tf32": prefill_flops / (prefill_local * 1e-3) / 1e12 / (0.5 * tf_peak),
+                         "tensor_peaks": f"bf16 {tf_peak:.1f} TFLOP/s ({peak_src}); tf32 (the MMAs' kind) "
+                                         f"{0.5 * tf_peak:.1f} = bf16 x 0.5, the nominal dense tf32:bf16 ratio"},
+            "varlen": varlen,
+            "decode_stream": dec_stream,
             "decode": None if args.only == "prefill" else {"us_per_step": 1000.0 * decode_max, "tokens_per_s": world * Bd * 1000.0 / decode_max,
                        "state_gbs": world * dec_bytes / (decode_max * 1e-3) / 1e9,
                        "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",

@@ -2,10 +2,12 @@
 //
 // Nothing here computes any part of the operator; it checks arguments, picks the kernel and
 // launches it on the caller's stream.
+#include <atomic>
 #include <mutex>
 
 #include "kda.h"
 #include "kda_internal.h"
+#include "kda_testing.h"
 
 namespace kda {
 
@@ -35,6 +37,8 @@ cudaError_t device_flags_ptr(unsigned int** out) {
     return cudaSuccess;
 }
 
+std::atomic<uint32_t> g_wait_polls{kDefaultWaitPolls};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool valid_dtype(kda_dtype d) { return d == KDA_BF16 || d == KDA_FP32; }
@@ -42,6 +46,8 @@ size_t dtype_size(kda_dtype d) { return d == KDA_FP32 ? 4 : 2; }
 bool supported_dim(int d) { return d == 64 || d == 128; }
 
 }  // namespace
+
+uint32_t consumer_wait_polls() { return g_wait_polls.load(std::memory_order_relaxed); }
 
 constexpr uint32_t kKnownOptions =
     KDA_OPT_SCALAR_GATE | KDA_OPT_L2NORM_QK | KDA_OPT_BETA_LOGITS | KDA_OPT_OUTPUT_NORM_GATE;
@@ -97,6 +103,7 @@ kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* lo
     a.beta_logits = (options & KDA_OPT_BETA_LOGITS) != 0;
     a.epilogue = (options & KDA_OPT_OUTPUT_NORM_GATE) != 0;
     a.out_gate = out_gate; a.norm_weight = norm_weight; a.norm_eps = norm_eps;
+    a.wait_polls = consumer_wait_polls();
     if (device_flags_ptr(&a.flags) != cudaSuccess) return KDA_ERR_CUDA;
 
     cudaError_t err;
@@ -238,5 +245,12 @@ const char* kda_status_string(kda_status status) {
 }
 
 uint32_t kda_version(void) { return (1u << 16) | 0u; }
+
+void kda_testing_set_wait_limit(int64_t polls) {
+    const uint32_t v = polls < 0 ? kda::kDefaultWaitPolls
+                                 : polls > static_cast<int64_t>(kda::kDefaultWaitPolls) ? kda::kDefaultWaitPolls
+                                                                                        : static_cast<uint32_t>(polls);
+    kda::g_wait_polls.store(v, std::memory_order_relaxed);
+}
 
 }  // extern "C"

@@ -12,13 +12,17 @@
 //       32 x 32 and 64 x 64 inverses with [[T1, 0], [-T2 A21 T1, T2]] on warp-level tensor-core
 //       tiles (mma.sync tf32, fp32 accumulation)
 //   W^T = (beta K e^G)^T T^T,  U^T = (beta V)^T T^T                MMA 2 (A operands in tensor memory)
-//   [Mt^T - Diag(e^{g_C}) | Qh^T - (Q e^G)^T] = -W^T [Kt | P^T]      MMA 3 (N = 192)
-//   [B^T | Uo^T] = U^T [Kt | P^T]                                    MMA 4 (N = 192)
+//   [Mt^T | Qh^T] = [Diag(e^{g_C}) | (Q e^G)^T] - W^T [Kt | P^T]     MMA 3 (N = 256, seeded accumulator)
+//   [B^T | Uo^T] = U^T [Kt | P^T]                                    MMA 4 (N = 256)
+// P enters the outputs' own terms (Uo = P U, Qh = Q e^G - P W), so it is carried as two tf32 parts,
+// P_hi = tf32(P) and P_lo = tf32(P - P_hi): the B operand of MMAs 3 and 4 is [Kt; P_hi; P_lo], and
+// the two halves of each output product are summed when read out.  This removes the largest rounding
+// term of the outputs (P rounded to tf32), about a third of their largest error.
 // Everything is formed transposed, with the key channel (or value column) as the tensor-memory lane:
 // the elementwise pass owns a channel and writes its operands straight into tensor memory, and each
 // record row goes from a lane's registers to the record in coalesced runs.  Every tcgen05 tf32 MMA
-// instruction costs about the same time for any N up to 192, so the products are grouped into few
-// wide instructions: 16 for MMA 1, 16 for MMA 2, 8 each for MMAs 3 and 4.
+// instruction costs about the same time for any N up to 192 (N = 256 about a third more), so the
+// products are grouped into few wide instructions: 16 for MMA 1, 16 for MMA 2, 8 each for MMAs 3 and 4.
 //
 // Decay factors: secondary chunking.  "일반 DPLR보다 줄어든 연산량" on the same page notes that with a
 // decay per channel the intra-chunk division is numerically delicate (a factor e^{-g} overflows) and
@@ -71,24 +75,27 @@ using wy::DV;
 constexpr int THREADS = 512;
 constexpr int TP = 68;  // row stride (floats) of the fp32 A and T tiles (conflict-free MMA fragment reads)
 constexpr float kSpanLimit = 80.f;  // largest log-decay span of a 16-row block kept in its MMA product
-constexpr uint32_t kWaitPolls = 1u << 26;
+constexpr uint32_t kWaitPolls = kDefaultWaitPolls;  // bound of the waits that drain work in flight
 
 // ---- shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_SQ = 0;         // q staging bf16 [64][128], two 64-channel boxes, 128-byte swizzle
 constexpr uint32_t OFF_SK = 16384;     // k staging bf16
-constexpr uint32_t OFF_SV = 32768;     // v staging bf16; later P in fp32 while strong-decay terms are added
-constexpr uint32_t OFF_G = 49152;      // log_alpha staging; then, fp32 at sw128_off(r, c, 64), the row factors
+constexpr uint32_t OFF_G = 32768;      // log_alpha staging; then, fp32 at sw128_off(r, c, 64), the row factors
                                        //   e^{g - a} -- or g itself when some channel decays strongly
-constexpr uint32_t OFF_Y = 81920;      // column tiles of MMA 1: tile R (rows 0 .. 16 R + 15, K e^{a_R - G}) at rows
+constexpr uint32_t OFF_Y = 65536;      // column tiles of MMA 1: tile R (rows 0 .. 16 R + 15, K e^{a_R - G}) at rows
                                        //   y_row(R) .. of one K-major tile, 160 rows x K c (128), sw128_off(n, c, 160)
-constexpr uint32_t OFF_KP = 163840;    // [Kt; P] K-major: rows n (Kt^T rows c 0..127, P rows t 128..191) x K s (64),
-                                       //   sw128_off(n, s, 192): B of MMAs 3 and 4
+constexpr uint32_t OFF_KP = 147456;    // [Kt; P_hi; P_lo] K-major: rows n (Kt^T rows c 0..127, P rows t 128..191 and
+                                       //   its rounding remainder 192..255) x K s (64), sw128_off(n, s, 256): B of
+                                       //   MMAs 3 and 4; K-block b at OFF_KP + 32768 b
 // per-channel factors of each 16-row block, until P is written over them (the P rows of each K-block):
 constexpr uint32_t OFF_FAC = OFF_KP + 16384;   // anchors a[4][128], e^{g_e - a}[4][128], e^{g_C - g_e}[4][128],
                                                //   e^{a}[4][128]  (g_e: g at the block's last row)
-constexpr uint32_t OFF_RHO = OFF_KP + 40960;   // e^{a_R - g_eI} [6][128] for block pairs R > I
-constexpr uint32_t OFF_XP = 212992;    // column sums of each 4-row group [16][128]
-constexpr uint32_t OFF_MISC = 221184;  // beta[2][64] (this task, the next), e^{g_C} [128], strong-decay channel
+constexpr uint32_t OFF_RHO = OFF_KP + 49152;   // e^{a_R - g_eI} [6][128] for block pairs R > I
+// v staging bf16: its two 64-channel boxes in the P_lo rows of the two K-blocks (the next task's v is
+// loaded once MMAs 3 and 4 are complete)
+constexpr uint32_t OFF_SV0 = OFF_KP + 24576;
+constexpr uint32_t OFF_SV1 = OFF_KP + 57344;
+constexpr uint32_t OFF_MISC = 212992;  // beta[2][64] (this task, the next), e^{g_C} [128], strong-decay channel
                                        //   masks [4 blocks][4 words]
 constexpr uint32_t MISC_BYTES = (128 + 128) * 4 + 64;
 constexpr uint32_t OFF_TASK = OFF_MISC + MISC_BYTES;  // three Task slots (this task, the next, the one after)
@@ -102,21 +109,24 @@ constexpr uint32_t OFF_A = OFF_Y;              // A fp32 [64][TP]
 constexpr uint32_t OFF_T32 = OFF_Y + 17408;    // T fp32 [64][TP]
 constexpr uint32_t OFF_TIMG = OFF_Y + 35840;   // T K-major rows r x K s (64), B of MMA 2
 constexpr uint32_t OFF_XS = OFF_Y + 52224;     // 32 x 32 fp32 scratch for the inverse
-constexpr uint32_t OFF_PF = OFF_SV;            // P fp32 [64][64] (16-byte chunks XOR-swizzled by row)
+constexpr uint32_t OFF_PF = OFF_Y + 56320;     // P fp32 [64][64] (16-byte chunks XOR-swizzled by row)
 // after MMA 2:
 constexpr uint32_t OFF_WT = OFF_Y;             // -W^T K-major rows j x K s (64), A of MMA 3
 constexpr uint32_t OFF_UT = OFF_Y + 32768;     // U^T K-major rows dv x K s (64), A of MMA 4
-// after MMAs 3 and 4: the record's Qh and Mt tiles, in the record's layout, for two bulk copies
-constexpr uint32_t OFF_STQ = OFF_Y;            // Qh, 32 KB
-constexpr uint32_t OFF_STM = OFF_Y + 32768;    // Mt, 64 KB
-static_assert(OFF_STM + 65536 <= OFF_XP, "record staging");
-static_assert(OFF_XS + 4096 <= OFF_KP && OFF_UT + 32768 <= OFF_KP, "tiles overlap [Kt; P]");
-static_assert(OFF_XP + 16 * 128 * 4 <= OFF_MISC, "group sums");
-static_assert(OFF_FAC + 16 * 128 * 4 <= OFF_KP + 24576 && OFF_RHO + 6 * 128 * 4 <= OFF_KP + 49152, "factors");
-static_assert(OFF_KP + 49152 <= OFF_XP, "[Kt; P]");
+// after MMAs 3 and 4: the record's [Mt; Qh] tile, in the record's layout, for one bulk copy (clear of
+// what the next task writes before it waits for the copy -- the group sums and the block factors -- and
+// of the v boxes it loads)
+constexpr uint32_t OFF_STG = OFF_Y;            // 96 KB
+// column sums of each 4-row group [16][128], in [Kt; P]'s Kt rows of K-block 1 (until Kt is written)
+constexpr uint32_t OFF_XP = OFF_KP + 32768;
+static_assert(OFF_PF + 16384 <= OFF_Y + 81920 && OFF_UT + 32768 <= OFF_KP, "post-MMA tiles overlap [Kt; P]");
+static_assert(OFF_XP >= OFF_STG + wy::REC_MQ_BYTES && OFF_XP + 16 * 128 * 4 <= OFF_KP + 32768 + 16384, "group sums");
+static_assert(OFF_STG + wy::REC_MQ_BYTES <= OFF_FAC, "record staging");
+static_assert(OFF_FAC + 16 * 128 * 4 <= OFF_SV0 && OFF_RHO + 6 * 128 * 4 <= OFF_SV1, "factors");
+static_assert(OFF_SV1 + 8192 <= OFF_MISC, "[Kt; P]");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 static_assert(OFF_TIMG % 1024 == 0 && OFF_WT % 1024 == 0 && OFF_UT % 1024 == 0 && OFF_Y % 1024 == 0 &&
-              OFF_KP % 1024 == 0, "swizzle atoms");
+              OFF_KP % 1024 == 0 && OFF_SV0 % 1024 == 0 && OFF_SV1 % 1024 == 0, "swizzle atoms");
 
 // first row of column tile R within the 160-row tile (tile R has 16 R + 16 rows)
 __host__ __device__ constexpr int y_row(int R) { return 8 * R * (R + 1); }
@@ -128,12 +138,19 @@ constexpr uint32_t TM_X = 0;      // [K; Q] rows scaled by e^{G - a}, 128 x 128,
 constexpr uint32_t TM_D1 = 128;   // MMA 1, 128 x 160: block R's columns at TM_D1 + y_row(R)
 constexpr uint32_t TM_BK = 320;   // (beta K e^G)^T, 128 (c) x 64 (s), A of MMA 2
 constexpr uint32_t TM_BV = 384;   // (beta V)^T, 128 (dv) x 64 (s), A of MMA 2
-constexpr uint32_t TM_QG = 448;   // (Q e^G)^T, 128 (j) x 64 (t): added to Qh^T when it is read out
+constexpr uint32_t TM_QG = 448;   // (Q e^G)^T, 128 (j) x 64 (t): copied into MMA 3's accumulator before it runs
 constexpr uint32_t TM_WT = 0;     // W^T, 128 x 64 (after MMA 1)
 constexpr uint32_t TM_UT = 64;    // U^T, 128 x 64
-constexpr uint32_t TM_DW = 0;     // MMA 3, 128 (j) x 192: -W^T Kt (i = 0..127), then -W^T P^T (t)   (after MMA 2)
-constexpr uint32_t TM_DU = 192;   // MMA 4, 128 (dv) x 192: B^T = U^T Kt, then Uo^T = U^T P^T
+constexpr uint32_t TM_DW = 0;     // MMA 3, 128 (j) x 256, seeded [Diag(e^{g_C}) | (Q e^G)^T | 0]: Mt^T, then Qh^T in
+                                  //   two parts (P_hi, P_lo)                                   (after MMA 2)
+constexpr uint32_t TM_DU = 256;   // MMA 4, 128 (dv) x 256: B^T, then Uo^T in two parts (P_hi, P_lo)
 constexpr uint32_t TM_COLS = 512;
+
+// Byte offset of element (t, i) of the fp32 P tile at OFF_PF: rows of 256 bytes, 16-byte chunk i / 4
+// XOR-swizzled with t % 16 so that a warp's rows do not share banks.
+__device__ __forceinline__ uint32_t pf_off(int t, int i) {
+    return static_cast<uint32_t>(t * 256 + ((((i >> 2) ^ (t & 15))) << 4) + ((i & 3) << 2));
+}
 
 __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
@@ -150,11 +167,6 @@ __device__ __forceinline__ float recip_approx(float x) {
     return y;
 }
 
-// Byte offset of element (t, i) of the fp32 P tile at OFF_PF: rows of 256 bytes, 16-byte chunk i / 4
-// XOR-swizzled with t % 16 so that a warp's rows do not share banks.
-__device__ __forceinline__ uint32_t pf_off(int t, int i) {
-    return static_cast<uint32_t>(t * 256 + ((((i >> 2) ^ (t & 15))) << 4) + ((i & 3) << 2));
-}
 
 // Byte offset of element (r, c) of a bf16 [64][128] tile loaded as two 64-channel boxes with the
 // 128-byte swizzle: box c / 64, row r at r * 128, 16-byte chunks permuted by XOR with r % 8.
@@ -343,7 +355,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const TG* __restrict__ beta, const TG* __restrict__ log_alpha_sg,
                   const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H,
-                  unsigned char* __restrict__ ws, unsigned int* flags, int beta_logits) {
+                  unsigned char* __restrict__ ws, unsigned int* flags, int beta_logits, uint32_t wait_polls) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;   // tensor-memory lane quadrant
     const int qr = warp >> 2;  // row block (elementwise pass) / column quarter (row pass, read-outs)
@@ -377,14 +389,21 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // Tile j (k, q, v, log_alpha) of a task into the staging buffers: one box covering all of the
     // tile's 128-byte column blocks (completion on bar_tma, whose expected byte count kStageBytes is
     // set once per task).  The four are issued by different warps.
-    constexpr int kLoads = SG ? 3 : 4;
+    // Boxes 0..2: k, q, log_alpha (issued by warps 0..2, SG: k, q); boxes 3, 4: the two 64-channel halves
+    // of v (into the P_lo rows of [Kt; P], so the next task's v is loaded only once MMAs 3 and 4 are done)
+    constexpr int kLoads = SG ? 2 : 3;
     auto load_box = [&](const Task& t, int j) {
-        const CUtensorMap* m = j == 0 ? &tm_k : j == 1 ? &tm_q : j == 2 ? &tm_v : &tm_g;
-        const uint32_t dst = j == 0 ? OFF_SK : j == 1 ? OFF_SQ : j == 2 ? OFF_SV : OFF_G + (sizeof(TG) == 4 ? 0u : 16384u);
+        if (j >= 3) {
+            tma_load_4d(sm + (j == 3 ? OFF_SV0 : OFF_SV1), &tm_v, 0, static_cast<int>(t.c0), j - 3, t.h, bar_tma);
+            return;
+        }
+        const CUtensorMap* m = j == 0 ? &tm_k : j == 1 ? &tm_q : &tm_g;
+        const uint32_t dst = j == 0 ? OFF_SK : j == 1 ? OFF_SQ : OFF_G + (sizeof(TG) == 4 ? 0u : 16384u);
         tma_load_4d(sm + dst, m, 0, static_cast<int>(t.c0), 0, t.h, bar_tma);
     };
 
     uint32_t loads_issued = 0;    // thread 0: staging loads issued (bar_tma phases)
+    bool v_pending = false;       // thread 0: the last phase's v boxes are not issued yet
     TaskWalker walker;            // the last thread's: it looks the tasks up
     constexpr int kWalker = THREADS - 1;
     if (tid == kWalker) {
@@ -404,6 +423,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0 && slots[0].id >= 0) {
         mbar_arrive_expect_tx(bar_tma, kStageBytes);
         for (int j = 0; j < kLoads; ++j) load_box(slots[0], j);
+        load_box(slots[0], 3);
+        load_box(slots[0], 4);
         ++loads_issued;
     }
     tc_fence_before_sync();
@@ -428,6 +449,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK);
     const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ);
     auto gf_at = [&](int r, int ch) -> float& { return *reinterpret_cast<float*>(sm + OFF_G + sw128_off(r, ch, 64)); };
+    // P[t][i .. i + 3] into its operand rows of [Kt; P_hi; P_lo]: P_hi = tf32(P) and the remainder
+    // P_lo = tf32(P - P_hi), so that the products with P carry its fp32 value (P enters Uo = P U and
+    // Qh = Q e^G - P W, the outputs' own terms)
+    auto put_p = [&](int t, int i, const float (&p)[4]) {
+        float hi[4], lo[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            hi[u] = to_tf32(p[u]);
+            lo[u] = to_tf32(p[u] - hi[u]);
+        }
+        *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + t, i, 256)) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(192 + t, i, 256)) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+    };
     const int rbq = 4 * qr;  // the elementwise pass's rows: 16 I + rbq .. + 3 of every block I
     // Byte offsets of (row, channel c) within a 128-byte row, for rows congruent to rbq + w mod 8: swf[w]
     // in the fp32 tiles (sw128_off), swb[w] in the bf16 staging tiles (bf16_sw_off, block of 64 channels
@@ -444,7 +478,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t swb0 = static_cast<uint32_t>(q4 >> 1) * 8192u + (static_cast<uint32_t>(4 * (q4 & 1) + (lane >> 3)) << 4) +
                           (static_cast<uint32_t>(lane & 7) << 1);
     const uint32_t colf = static_cast<uint32_t>(q4) * 8192u;  // channel block of c in a 64-row fp32 tile
+    // the v box of channel c (two separate 8 KB boxes) replaces the 64-channel block offset of swb
+    const uint32_t vbox = (q4 >> 1) ? OFF_SV1 : OFF_SV0;
+    const uint32_t vblk = static_cast<uint32_t>(q4 >> 1) * 8192u;
 
+    uint32_t mma_issued = 0;  // thread 0: bit k - 1 set once MMA k of the current task is committed
+    uint32_t cur_par = 0;     // phase parity of the current task's barriers
     int cur = 0;  // slot of this task in the ring of three
     for (uint32_t it = 0;; ++it, cur = cur == 2 ? 0 : cur + 1) {  // `it`: tasks taken; phase parities follow from it
         const int nxt = cur == 2 ? 0 : cur + 1, aft = nxt == 2 ? 0 : nxt + 1;
@@ -454,7 +493,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         unsigned char* rec = tk.rec;
         const uint32_t par = it & 1;
         const float* s_beta = s_beta2 + 64 * par;
-        failed = !mbar_wait(bar_tma, par, kWaitPolls);
+        cur_par = par;
+        mma_issued = 0;
+        failed = !mbar_wait(bar_tma, par, wait_polls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
 
@@ -535,7 +576,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (I == 3) s_gam[c] = __expf(gl[3]);
             }
         }
-        if (tid == 0) bulk_wait_read();  // the previous record's Qh and Mt tiles have left shared memory
+        if (tid == 0) bulk_wait_read();  // the previous record's [Mt; Qh] tile has left shared memory
         const bool any_strong = __syncthreads_or(strong != 0);
 
         // ---- 3: per element (row i, channel c): the row factor e^{g_i - a} (for the row pass; g itself when
@@ -560,7 +601,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint32_t ob = swb[w] + i * 128;  // (i, c) in the bf16 staging tiles
                     float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK + ob));
                     float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ + ob));
-                    float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SV + ob));
+                    float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + vbox + (ob - vblk)));
                     if (PRO) { kv *= s_rn[i]; qv *= s_rn[64 + i]; }
                     if (!live) { kv = 0.f; qv = 0.f; vv = 0.f; }
                     const float b = s_beta[i];
@@ -588,7 +629,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     bv[w] = to_tf32(b * vv);
                     qg[w] = qv * Gm;
                 }
-                *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 192)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+                *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
                 tmem_st4(tq + TM_BK + 16 * I + rbq, bk);
                 tmem_st4(tq + TM_BV + 16 * I + rbq, bv);
                 tmem_st4(tq + TM_QG + 16 * I + rbq, qg);
@@ -647,8 +688,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mma_tf32_ts(tmem + TM_D1, tmem + TM_X + 8 * kk, by + (((kk >> 2) * 160 * 128 + (kk & 3) * 32) >> 4), id1,
                             kk > 0);
             mma_commit(bar_m1);
+            mma_issued |= 1u;
         }
-        failed = !mbar_wait(bar_m1, par, kWaitPolls);
+        failed = !mbar_wait(bar_m1, par, wait_polls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
         {   // lane rows 0..63 -> A (beta-scaled, strictly lower, fp32); 64..127 -> P (lower with the
@@ -681,8 +723,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                         for (int u = 0; u < 4; ++u) p[u] = (i0 + k4 + u) <= row ? x[k4 + u] : 0.f;
                         if (!any_strong)
-                            *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + row, i0 + k4, 192)) =
-                                make_float4(to_tf32(p[0]), to_tf32(p[1]), to_tf32(p[2]), to_tf32(p[3]));
+                            put_p(row, i0 + k4, p);
                         else
                             *reinterpret_cast<float4*>(sm + OFF_PF + pf_off(row, i0 + k4)) = make_float4(p[0], p[1], p[2], p[3]);
                     }
@@ -691,10 +732,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (isq && qr > Rl) {  // P above the row's block: zeros
 #pragma unroll
                 for (int k4 = 0; k4 < 16; k4 += 4) {
-                    if (!any_strong)
-                        *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + row, 16 * qr + k4, 192)) =
-                            make_float4(0.f, 0.f, 0.f, 0.f);
-                    else
+                    if (!any_strong) {
+                        const float z[4] = {0.f, 0.f, 0.f, 0.f};
+                        put_p(row, 16 * qr + k4, z);
+                    } else
                         *reinterpret_cast<float4*>(sm + OFF_PF + pf_off(row, 16 * qr + k4)) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
@@ -741,8 +782,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const float4 p = *reinterpret_cast<const float4*>(sm + OFF_PF + pf_off(t, i8 + 4 * h));
-                    *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + t, i8 + 4 * h, 192)) =
-                        make_float4(to_tf32(p.x), to_tf32(p.y), to_tf32(p.z), to_tf32(p.w));
+                    const float pv[4] = {p.x, p.y, p.z, p.w};
+                    put_p(t, i8 + 4 * h, pv);
                 }
             }
         }
@@ -751,6 +792,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (tid == 0 && tn.id >= 0) {
             mbar_arrive_expect_tx(bar_tma, kStageBytes);
             ++loads_issued;
+            v_pending = true;  // v once MMAs 3 and 4 have read the P_lo rows it lands in
         }
         __syncthreads();
         if (lane == 0 && warp < kLoads && tn.id >= 0) load_box(tn, warp);
@@ -785,11 +827,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mma_tf32_ts(tmem + TM_UT, tmem + TM_BV + 8 * kk, b, id2, kk > 0);
             }
             mma_commit(bar_m2);
+            mma_issued |= 2u;
         }
         if (tid == kWalker) slots[aft] = walker.next();  // while MMA 2 runs: the task after the next
-        failed = !mbar_wait(bar_m2, par, kWaitPolls);
+        failed = !mbar_wait(bar_m2, par, wait_polls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
+        float qg[16];  // (Q e^G)^T of lane c, tokens 16 qr .. +15: moved into MMA 3's accumulator below
         {   // -W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..)
             float x[32];
             const bool isw = qr < 2;
@@ -800,33 +844,52 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int e4 = 0; e4 < 32; e4 += 4)
                 *reinterpret_cast<float4*>(tile + sw128_off(c, 32 * (qr & 1) + e4, 128)) =
                     make_float4(to_tf32(sgn * x[e4]), to_tf32(sgn * x[e4 + 1]), to_tf32(sgn * x[e4 + 2]), to_tf32(sgn * x[e4 + 3]));
+            tmem_ld16(tq + TM_QG + 16 * qr, qg);
+        }
+        tc_fence_before_sync();
+        __syncthreads();  // W^T, U^T and (Q e^G)^T are read: MMA 3's accumulator may be filled over them
+        tc_fence_after_sync();
+        {   // MMA 3's accumulator <- [Diag(e^{g_C}) | (Q e^G)^T | 0] (lane j = c): the MMA then adds -W^T [Kt; P]^T
+            float d[32];
+            const float gam = s_gam[c];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) d[e] = (32 * qr + e == c) ? gam : 0.f;
+            tmem_st32(tq + TM_DW + 32 * qr, d);
+            tmem_st16(tq + TM_DW + 128 + 16 * qr, qg);
+            float z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) z[e] = 0.f;
+            tmem_st16(tq + TM_DW + 192 + 16 * qr, z);
+            tmem_st_wait();
         }
         fence_async_smem();
         tc_fence_before_sync();
         __syncthreads();
 
-        // ---- MMA 3: [-W^T Kt | -W^T P^T] (= Mt^T - Diag(e^{g_C}) | Qh^T - (Q e^G)^T);  MMA 4: [U^T Kt | U^T P^T]
-        //      (= B^T | Uo^T).  M=128, N=192 ([Kt; P] rows), K=64 (tokens s); A and B in shared memory.
+        // ---- MMA 3: [Diag(e^{g_C}) | (Q e^G)^T | 0] - W^T [Kt; P_hi; P_lo]^T = [Mt | Qh^T split in two halves];
+        //      MMA 4: U^T [Kt; P_hi; P_lo]^T = [B^T | Uo^T split in two halves].  M=128, N=256, K=64 (tokens s);
+        //      A and B in shared memory.
         if (tid == 0) {
             tc_fence_after_sync();
             const uint64_t aw = sw128_desc(sbase + OFF_WT, 16, 1024);
             const uint64_t au = sw128_desc(sbase + OFF_UT, 16, 1024);
             const uint64_t bkp = sw128_desc(sbase + OFF_KP, 16, 1024);
-            constexpr uint32_t id3 = idesc_tf32(128, 192, false, false);
+            constexpr uint32_t id3 = idesc_tf32(128, 256, false, false);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)
                 mma_tf32(tmem + TM_DU, au + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                         bkp + (((kk >> 2) * 24576 + (kk & 3) * 32) >> 4), id3, kk > 0);
+                         bkp + (((kk >> 2) * 32768 + (kk & 3) * 32) >> 4), id3, kk > 0);
             mma_commit(bar_m4);
 #pragma unroll
-            for (int kk = 0; kk < C / 8; ++kk)
+            for (int kk = 0; kk < C / 8; ++kk)  // onto the seeded accumulator
                 mma_tf32(tmem + TM_DW, aw + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                         bkp + (((kk >> 2) * 24576 + (kk & 3) * 32) >> 4), id3, kk > 0);
+                         bkp + (((kk >> 2) * 32768 + (kk & 3) * 32) >> 4), id3, 1);
             mma_commit(bar_m3);
+            mma_issued |= 12u;
         }
         // a timed-out wait here is acted on at the end of the task (the read-outs below then only
         // write garbage into this task's own record)
-        bool late = !mbar_wait(bar_m4, par, kWaitPolls);
+        bool late = !mbar_wait(bar_m4, par, wait_polls);
         tc_fence_after_sync();
         {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record
             float x[32];
@@ -850,46 +913,61 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 gb[(4 * qr + s8) * 128 + c] = make_uint4(w[0], w[1], w[2], w[3]);
             }
             reinterpret_cast<signed char*>(rec + wy::REC_BEXP)[qr * 128 + c] = static_cast<signed char>(ex);
-            float y[16];
+            float y[16], yl[16];  // U^T P_hi^T + U^T P_lo^T
             tmem_ld16(tq + TM_DU + 128 + 16 * qr, y);
+            tmem_ld16(tq + TM_DU + 192 + 16 * qr, yl);
             float4* gu = reinterpret_cast<float4*>(rec + wy::REC_UO);
 #pragma unroll
             for (int s4 = 0; s4 < 4; ++s4)
-                gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4], y[4 * s4 + 1], y[4 * s4 + 2], y[4 * s4 + 3]);
+                gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4] + yl[4 * s4], y[4 * s4 + 1] + yl[4 * s4 + 1],
+                                                          y[4 * s4 + 2] + yl[4 * s4 + 2], y[4 * s4 + 3] + yl[4 * s4 + 3]);
         }
-        late |= !mbar_wait(bar_m3, par, kWaitPolls);
+        late |= !mbar_wait(bar_m3, par, wait_polls);
         tc_fence_after_sync();
-        {   // Mt (lane j = c, rows i = 32 qr ..) and Qh (lane j, tokens t = 16 qr ..) into their record tiles
-            // in shared memory (for each i or t the warp's 32 lanes write one 128-byte row), then two bulk
-            // copies.  The [Kt; P] and W^T, U^T tiles under them are dead: MMAs 3 and 4 are complete.
+        {   // Mt (lane j = c, rows i = 32 qr ..) and Qh (lane j, tokens t = 16 qr ..) into the record's [Mt; Qh]
+            // tile in shared memory (for each row the warp's 32 lanes write one 128-byte run), then one bulk
+            // copy.  The [Kt; P] and W^T, U^T tiles under it are dead: MMAs 3 and 4 are complete.
             float x[32];
             tmem_ld32(tq + TM_DW + 32 * qr, x);
-            const float gam = s_gam[c];
-            unsigned char* stm = sm + OFF_STM + q4 * 16384 + ((lane & 3) << 2);
+            unsigned char* stg = sm + OFF_STG + q4 * wy::REC_MQ_KBLOCK + ((lane & 3) << 2);  // K-block of channel c
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const int i = 32 * qr + e;  // row i of K-block q4 of Mt; its 16-byte chunks permuted by i % 8 = e % 8
-                *reinterpret_cast<float*>(stm + i * 128 + (((lane >> 2) ^ (e & 7)) << 4)) = to_tf32(x[e] + (i == c ? gam : 0.f));
+                const int i = 32 * qr + e;  // row i; its 16-byte chunks permuted by i % 8 = e % 8
+                *reinterpret_cast<float*>(stg + i * 128 + (((lane >> 2) ^ (e & 7)) << 4)) = to_tf32(x[e]);
             }
-            float y[16], sd[16];
+            float y[16], sd[16];  // the hi and lo halves of Qh^T
             tmem_ld16(tq + TM_DW + 128 + 16 * qr, y);
-            tmem_ld16(tq + TM_QG + 16 * qr, sd);
+            tmem_ld16(tq + TM_DW + 192 + 16 * qr, sd);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                *reinterpret_cast<float*>(sm + OFF_STQ + sw128_off(16 * qr + e, c, 64)) = to_tf32(y[e] + sd[e]);
+            for (int e = 0; e < 16; ++e) {
+                const int n = 128 + 16 * qr + e;  // row of token t = 16 qr + e
+                *reinterpret_cast<float*>(stg + n * 128 + (((lane >> 2) ^ (e & 7)) << 4)) = to_tf32(y[e] + sd[e]);
+            }
         }
         fence_async_smem();
         tc_fence_before_sync();
         if (__syncthreads_or(late)) { failed = true; break; }
         if (tid == 0) {
-            bulk_store(rec + wy::REC_M, sm + OFF_STM, 65536);
-            bulk_store(rec + wy::REC_Q, sm + OFF_STQ, 32768);
+            if (v_pending) {
+                load_box(tn, 3);
+                load_box(tn, 4);
+                v_pending = false;
+            }
+            bulk_store(rec + wy::REC_MQ, sm + OFF_STG, wy::REC_MQ_BYTES);
             bulk_commit();
         }
     }
 
     if (failed && tid == 0) {
-        // leave no copy into this CTA's shared memory behind: wait (bounded) for the last staging load
+        // leave no copy into this CTA's shared memory and no MMA writing its tensor memory behind: wait
+        // (bounded, with the default limit) for the last staging load and for every MMA of the task
+        // that was committed
+        for (int k = 0; k < 4; ++k)
+            if (mma_issued & (1u << k)) mbar_wait(bar_m1 + k, cur_par, kWaitPolls);
+        if (v_pending) {  // complete the pending phase (its other boxes are in flight), now that no MMA reads P_lo
+            load_box(slots[cur == 2 ? 0 : cur + 1], 3);
+            load_box(slots[cur == 2 ? 0 : cur + 1], 4);
+        }
         if (loads_issued > 0) mbar_wait(bar_tma, (loads_issued - 1) & 1, kWaitPolls);
         raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
     }
@@ -920,7 +998,7 @@ cudaError_t launch_prep(const ChunkArgs& a) {
     constexpr CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     if (!tma_encode_blocks(&mq, a.q, bf, 2, DK, H, T, 64, C, sw) ||
         !tma_encode_blocks(&mk, a.k, bf, 2, DK, H, T, 64, C, sw) ||
-        !tma_encode_blocks(&mv, a.v, bf, 2, DV, H, T, 64, C, sw) ||
+        !tma_encode_blocks(&mv, a.v, bf, 2, DV, H, T, 64, C, sw, 1) ||
         (!SG && !tma_encode_blocks(&mg, a.log_alpha, gdt, sizeof(TG), DK, H, T, gblk, C, sw)))
         return cudaErrorInvalidValue;
     if (SG) mg = mq;  // not read
@@ -933,7 +1011,7 @@ cudaError_t launch_prep(const ChunkArgs& a) {
     kern<<<grid, THREADS, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, static_cast<const TG*>(a.beta),
                                                   SG ? static_cast<const TG*>(a.log_alpha) : nullptr, a.cu_seqlens,
                                                   a.T_total, a.N, a.H, static_cast<unsigned char*>(a.workspace),
-                                                  a.flags, a.beta_logits ? 1 : 0);
+                                                  a.flags, a.beta_logits ? 1 : 0, a.wait_polls);
     return cudaGetLastError();
 }
 

@@ -49,7 +49,7 @@ constexpr int THREADS = 320;
 constexpr int DATA_THREADS = 256;
 constexpr int LOADER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr uint32_t kWaitPolls = 1u << 26;
+constexpr uint32_t kWaitPolls = kDefaultWaitPolls;  // bound of the waits that drain work in flight
 
 constexpr int DVH = 64;                  // value columns per CTA
 constexpr uint32_t STAGE_BYTES = 98304;  // Mt tile (64 KB) + Qh tile (32 KB)
@@ -73,9 +73,9 @@ constexpr uint32_t TM_COLS = 512;
 
 // Bounded wait (polls and wall time) that also gives up when another role has flagged an abort; a
 // timeout flags one.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t polls) {
     WaitBudget budget;
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    for (uint32_t i = 0; i < polls; ++i) {
         if (mbar_poll(bar, parity)) return true;
         if ((i & 255u) == 255u && *abort) return false;
         if (budget.expired()) break;
@@ -147,7 +147,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                   const int32_t* __restrict__ cu_seqlens, int64_t T_total, int N, int H, void* __restrict__ o_ptr,
                   int o_is_f32, float* final_state, unsigned int* flags, const void* __restrict__ out_gate,
                   int gate_is_f32, const float* __restrict__ norm_weight, float norm_eps, int nseg,
-                  float* __restrict__ s_mid, float* __restrict__ s0_copy) {
+                  float* __restrict__ s_mid, float* __restrict__ s0_copy, const int32_t* __restrict__ order,
+                  uint32_t wait_polls) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -165,7 +166,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
     const int seg = SONLY ? 0 : static_cast<int>((blockIdx.x >> 1) % nseg);
     const int unit = static_cast<int>((blockIdx.x >> 1) / (SONLY ? 1 : nseg));
     const int h = unit % H;
-    const int n = unit / H;
+    const int n = order ? order[unit / H] : unit / H;  // longest sequences first when an order is given
     int64_t t0, t1;
     if (!wy::seq_bounds(cu_seqlens, T_total, N, n, t0, t1)) {
         if (tid == 0 && seg == 0 && !SONLY) raise_flag(flags, KDA_DEVFLAG_CU_SEQLENS);
@@ -267,7 +268,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
                     mbar_arrive_peer(peer_addr(pbar, static_cast<uint32_t>(half ^ 1)));
                     bool got = false;
                     WaitBudget budget;
-                    for (uint32_t i = 0; i < kWaitPolls && !got; ++i) {
+                    for (uint32_t i = 0; i < wait_polls && !got; ++i) {
                         got = mbar_try_cluster(pbar, (c >> 1) & 1);
                         if (!got && (((i & 255u) == 255u && *abort) || budget.expired())) break;
                     }
@@ -330,7 +331,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             // O_{c-2} is written to memory
             float ox[16];
             if (c >= 2) {  // (SONLY: odone marks the state product of the chunk, which freed the buffer)
-                ok = wait_or_abort(odone + (c & 1), ((c - 2) >> 1) & 1, abort);
+                ok = wait_or_abort(odone + (c & 1), ((c - 2) >> 1) & 1, abort, wait_polls);
                 if (!ok) break;
                 tc_fence_after_sync();
                 if (!SONLY) tmem_ld16_x2<16>(tq + TM_O + 64 * (c & 1) + 32 * g, ox);
@@ -365,7 +366,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             }
         }
         for (int c = nc - 2 < 0 ? 0 : nc - 2; c < nc && ok; ++c) {
-            ok = wait_or_abort(odone + (c & 1), (c >> 1) & 1, abort);
+            ok = wait_or_abort(odone + (c & 1), (c >> 1) & 1, abort, wait_polls);
             if (!ok) break;
             tc_fence_after_sync();
             if (SONLY) continue;
@@ -387,21 +388,20 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             int issued = 0;
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
-                if (c >= 2 && !wait_or_abort(empty + s, ((c - 2) >> 1) & 1, abort)) break;
+                if (c >= 2 && !wait_or_abort(empty + s, ((c - 2) >> 1) & 1, abort, wait_polls)) break;
                 const unsigned char* rec = ws + (static_cast<size_t>(slot0 + c) * H + h) * wy::REC_BYTES;
                 unsigned char* stage = sm + (s ? OFF_STAGE1 : OFF_STAGE0);
                 mbar_arrive_expect_tx(full + s, SONLY ? 65536 : STAGE_BYTES);  // SONLY: Mt alone
 #pragma unroll
-                for (int b = 0; b < 4; ++b) bulk_load(stage + 16384 * b, rec + wy::REC_M + 16384 * b, 16384, full + s);
-                if (!SONLY) {
-#pragma unroll
-                    for (int b = 0; b < 2; ++b)
-                        bulk_load(stage + 65536 + 16384 * b, rec + wy::REC_Q + 16384 * b, 16384, full + s);
+                for (int b = 0; b < 4; ++b) {  // K-block b of the record's [Mt; Qh] tile: Mt rows, then Qh rows
+                    const unsigned char* kb = rec + wy::REC_MQ + wy::REC_MQ_KBLOCK * b;
+                    bulk_load(stage + 16384 * b, kb, 16384, full + s);
+                    if (!SONLY) bulk_load(stage + 65536 + 8192 * b, kb + 16384, 8192, full + s);
                 }
                 if (c + 3 < nc) {  // the record three chunks ahead into L2 (SONLY: Mt and B)
                     const unsigned char* r3 = ws + (static_cast<size_t>(slot0 + c + 3) * H + h) * wy::REC_BYTES;
                     for (uint32_t off = 0; off < wy::REC_BYTES; off += 16384)
-                        if (!SONLY || off < wy::REC_Q || (off >= wy::REC_B && off < wy::REC_UO) || off >= wy::REC_BEXP)
+                        if (!SONLY || off < wy::REC_UO || off >= wy::REC_BEXP)
                             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(r3 + off),
                                          "r"(wy::REC_BYTES - off < 16384u ? wy::REC_BYTES - off : 16384u)
                                          : "memory");
@@ -423,9 +423,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
             int committed = 0;
             for (int c = 0; c < nc; ++c) {
                 const int s = c & 1;
-                if (!wait_or_abort(full + s, (c >> 1) & 1, abort)) break;
-                if (!wait_or_abort(sinit + s, (c >> 1) & 1, abort)) break;
-                if (c >= 1 && !wait_or_abort(chain, (c - 1) & 1, abort)) break;
+                if (!wait_or_abort(full + s, (c >> 1) & 1, abort, wait_polls)) break;
+                if (!wait_or_abort(sinit + s, (c >> 1) & 1, abort, wait_polls)) break;
+                if (c >= 1 && !wait_or_abort(chain, (c - 1) & 1, abort, wait_polls)) break;
                 tc_fence_after_sync();
                 const uint32_t st = sbase + (s ? OFF_STAGE1 : OFF_STAGE0);
                 const uint64_t bm = sw128_desc(st, 16, 1024);          // Mt, K-major rows i
@@ -464,11 +464,36 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char*
     if (EPI) cluster_sync_all();  // neither half leaves while the other may still write into it
 }
 
+// The sequences ranked by length, longest first (ties by index): order[rank] = sequence.  One CTA; thread
+// i counts the sequences that go before sequence i.  Malformed cu_seqlens (caught by the scan) only
+// spoil the order, which stays a permutation.
+__global__ void __launch_bounds__(1024) seq_order_kernel(const int32_t* __restrict__ cu, int N,
+                                                         int32_t* __restrict__ order) {
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        const int64_t Li = static_cast<int64_t>(cu[i + 1]) - cu[i];
+        int rank = 0;
+        for (int j = 0; j < N; ++j) {
+            const int64_t Lj = static_cast<int64_t>(cu[j + 1]) - cu[j];
+            rank += (Lj > Li || (Lj == Li && j < i)) ? 1 : 0;
+        }
+        order[rank] = i;
+    }
+}
+
 }  // namespace
 
-size_t chunk_scan_state_bytes(int N, int H) {  // s_mid and the copy of S_0, fp32 [N, H, dk, dv] each
-    return 2 * static_cast<size_t>(N) * static_cast<size_t>(H) * DK * DV * sizeof(float);
+// the scan's part of the workspace: s_mid and the copy of S_0, fp32 [N, H, dk, dv] each, then the
+// longest-first sequence order, int32 [N] (padded to 16 bytes)
+size_t chunk_scan_state_bytes(int N, int H) {
+    return 2 * static_cast<size_t>(N) * static_cast<size_t>(H) * DK * DV * sizeof(float) +
+           ((static_cast<size_t>(N) * sizeof(int32_t) + 15) & ~static_cast<size_t>(15));
 }
+
+namespace {
+// Longest-first ordering is used for packed batches of at most this many sequences (the ranking is
+// quadratic in N; beyond it the scan keeps the batch order).
+constexpr int kOrderMaxSeqs = 16384;
+}  // namespace
 
 cudaError_t launch_chunk_scan(const ChunkArgs& a) {
     CUtensorMap mo;
@@ -481,6 +506,13 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
     float* s_mid = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) +
                                             static_cast<size_t>(wy::num_slots(a.T_total, a.N)) * a.H * wy::REC_BYTES);
     float* s0_copy = s_mid + static_cast<size_t>(a.N) * a.H * DK * DV;
+    int32_t* order = nullptr;
+    if (a.cu_seqlens && a.N > 1 && a.N <= kOrderMaxSeqs) {
+        order = reinterpret_cast<int32_t*>(s0_copy + static_cast<size_t>(a.N) * a.H * DK * DV);
+        seq_order_kernel<<<1, 1024, 0, a.stream>>>(a.cu_seqlens, a.N, order);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     const int o32 = f32 ? 1 : 0, g32 = a.dtype_qkv == KDA_FP32 ? 1 : 0;
     // Intra-sequence split when there are few (sequence, head) units: the scan is then bound by each
     // sequence's chain of chunks, not by the record stream.  With more units the CTAs already pull
@@ -499,7 +531,7 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
         if (err != cudaSuccess) return err;
         chunk_scan_kernel<false, true><<<static_cast<unsigned>(units * 2), THREADS, SMEM_BYTES, a.stream>>>(
             mo, ws, a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o, o32, a.final_state, a.flags, nullptr, 0,
-            nullptr, 0.f, 1, s_mid, s0_copy);
+            nullptr, 0.f, 1, s_mid, s0_copy, order, a.wait_polls);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
@@ -510,7 +542,7 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
         if (err != cudaSuccess) return err;
         chunk_scan_kernel<false, false><<<blocks, THREADS, SMEM_BYTES, a.stream>>>(
             mo, ws, a.initial_state, a.cu_seqlens, a.T_total, a.N, a.H, a.o, o32, a.final_state, a.flags, nullptr, 0,
-            nullptr, 0.f, nseg, s_mid, s0_copy);
+            nullptr, 0.f, nseg, s_mid, s0_copy, order, a.wait_polls);
         return cudaGetLastError();
     }
     err = cudaFuncSetAttribute(chunk_scan_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -529,7 +561,7 @@ cudaError_t launch_chunk_scan(const ChunkArgs& a) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, chunk_scan_kernel<true, false>, mo, ws, a.initial_state, a.cu_seqlens, a.T_total,
                               a.N, a.H, a.o, o32, a.final_state, a.flags, a.out_gate, g32, a.norm_weight, a.norm_eps,
-                              nseg, s_mid, s0_copy);
+                              nseg, s_mid, s0_copy, order, a.wait_polls);
 }
 
 }  // namespace kda

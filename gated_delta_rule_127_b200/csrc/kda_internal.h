@@ -32,6 +32,7 @@ struct ChunkArgs {
     const void* out_gate; // [T_total, H, dv], dtype_qkv
     const float* norm_weight;  // [dv]
     float norm_eps;
+    uint32_t wait_polls;  // polls before a consumer-side bounded wait gives up (consumer_wait_polls())
 };
 
 struct DecodeArgs {
@@ -61,6 +62,12 @@ struct DecodeArgs {
 inline bool chunk_tc_path(int64_t T_total, kda_dtype dtype_qkv, int dk, int dv) {
     return dtype_qkv == KDA_BF16 && dk == 128 && dv == 128 && T_total > 0 && T_total < (int64_t(1) << 31);
 }
+
+// Polls before a bounded wait of a consumer (a role waiting for another role's data) gives up:
+// kDefaultWaitPolls unless kda_testing_set_wait_limit changed it.  Waits that drain work already in
+// flight on an abort keep kDefaultWaitPolls.  Either way each wait also ends after 2 s of wall time.
+constexpr uint32_t kDefaultWaitPolls = 1u << 26;
+uint32_t consumer_wait_polls();
 
 // Each launcher returns cudaSuccess or the launch error.
 cudaError_t launch_decode(const DecodeArgs& a);

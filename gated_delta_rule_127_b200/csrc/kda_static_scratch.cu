@@ -10,7 +10,7 @@ namespace kda {
 namespace {
 
 // KDA_STATIC_SCRATCH_BYTES = 32 MiB: the chunk records (160.5 KB per 64-token chunk slot and head) and the
-// scan's two state arrays (128 KB per sequence and head) of calls up to that size.
+// scan's two state arrays (128 KB per sequence and head) and sequence order of calls up to that size.
 // Reserved on each device when the library's device code is loaded there; never allocated by a call.
 __device__ __align__(256) unsigned char g_static_scratch[KDA_STATIC_SCRATCH_BYTES];
 

@@ -41,14 +41,16 @@ inline bool tma_encode_thd(CUtensorMap* m, const void* base, CUtensorMapDataType
 // strides {H d, blk, d} elements (not increasing, which the encoder accepts), so one box
 // {blk, box_tokens, d / blk, 1} lands in shared memory block after block, [block][token][blk channels]
 // -- with a 128-byte swizzle and blk * esize = 128 the layout of d / blk separate {blk, 1, box_tokens}
-// boxes of the 3-D view, in one copy.
+// boxes of the 3-D view, in one copy.  box_blocks (0: all d / blk) narrows the box to that many blocks,
+// for a tile loaded block by block.
 inline bool tma_encode_blocks(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, uint64_t d,
-                              uint64_t H, uint64_t T, uint32_t blk, uint32_t box_tokens, CUtensorMapSwizzle swz) {
+                              uint64_t H, uint64_t T, uint32_t blk, uint32_t box_tokens, CUtensorMapSwizzle swz,
+                              uint32_t box_blocks = 0) {
     auto fn = tma_encode_fn();
     if (!fn || d % blk != 0) return false;
     const cuuint64_t dims[4] = {blk, T, d / blk, H};
     const cuuint64_t strides[3] = {H * d * esize, blk * esize, d * esize};
-    const cuuint32_t box[4] = {blk, box_tokens, static_cast<cuuint32_t>(d / blk), 1};
+    const cuuint32_t box[4] = {blk, box_tokens, box_blocks ? box_blocks : static_cast<cuuint32_t>(d / blk), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;

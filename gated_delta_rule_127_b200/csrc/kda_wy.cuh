@@ -11,11 +11,12 @@
 // computed in parallel; the scan then needs one dk x dk x dv and one C x dk x dv product per chunk.
 //
 // Record of one (chunk, head), REC_BYTES bytes, fp32:
-//   REC_M  Mt as the scan's B operand (K = key channel j, N = key channel i), K-major with the 128-byte
-//          swizzle: four 32-channel K-blocks of 128 rows x 128 bytes; element (i, j) at
-//          sw128_off(i, j, 128).  Rounded to tf32.
-//   REC_Q  Qh as the scan's B operand (K = j, N = token t): four K-blocks of 64 rows x 128 bytes;
-//          element (t, j) at sw128_off(t, j, 64).  Rounded to tf32.
+//   REC_MQ [Mt; Qh] as one B operand of the scan (K = key channel j; N = key channel i for the 128 Mt
+//          rows, then token t for the 64 Qh rows), K-major with the 128-byte swizzle: four 32-channel
+//          K-blocks of 192 rows x 128 bytes; Mt element (i, j) at sw128_off(i, j, 192), Qh element
+//          (t, j) at sw128_off(128 + t, j, 192).  Rounded to tf32.  One tile, so that the chunk-local
+//          kernel writes it with one bulk copy; the scan loads each K-block's Mt rows and Qh rows as
+//          separate operand tiles (a row's swizzle depends only on row % 8, the same in both).
 //   REC_B  B transposed, in fp16 with a power-of-two scale per 32 rows and value column, interleaved
 //          by eight: element (i, dv) is B[i][dv] * 2^-e at half index (i / 8) * 1024 + dv * 8 + i % 8,
 //          so thread dv reading 16 bytes at uint4 number (i / 8) * 128 + dv gets rows i..i+7 and a
@@ -38,8 +39,9 @@ namespace wy {
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DV = 128;
-constexpr uint32_t REC_M = 0;
-constexpr uint32_t REC_Q = 65536;
+constexpr uint32_t REC_MQ = 0;
+constexpr uint32_t REC_MQ_BYTES = 98304;
+constexpr uint32_t REC_MQ_KBLOCK = 24576;  // bytes of one 32-channel K-block (192 rows)
 constexpr uint32_t REC_B = 98304;
 constexpr uint32_t REC_UO = 131072;
 constexpr uint32_t REC_BEXP = 163840;

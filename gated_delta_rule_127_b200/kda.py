@@ -14,7 +14,8 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
-HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "kda.h")
+INCLUDE_DIR = os.path.join(os.path.dirname(_HERE), "include")
+HEADER_PATH = os.path.join(INCLUDE_DIR, "kda.h")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_DEVICE_CHECK = range(6)
 KDA_BF16, KDA_FP32 = 0, 1
@@ -63,15 +64,20 @@ def load_library() -> ctypes.CDLL:
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
     lib.kda_version.restype = ctypes.c_uint32
+    lib.kda_testing_set_wait_limit.argtypes = [i64]
+    lib.kda_testing_set_wait_limit.restype = None
     _lib = lib
     return lib
 
 
 def header_symbols():
-    """Names of the entry points include/kda.h declares."""
-    with open(HEADER_PATH) as f:
-        text = f.read()
-    return re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", text)
+    """Names of the entry points the headers under include/ declare."""
+    names = []
+    for fn in sorted(os.listdir(INCLUDE_DIR)):
+        if fn.endswith(".h"):
+            with open(os.path.join(INCLUDE_DIR, fn)) as f:
+                names += re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", f.read())
+    return names
 
 
 def status_string(status: int) -> str:
@@ -84,6 +90,12 @@ def kda_status_string(status: int) -> str:
 
 def kda_version() -> int:
     return int(load_library().kda_version())
+
+
+def kda_testing_set_wait_limit(polls: int) -> None:
+    """Test hook (include/kda_testing.h): polls >= 0 bounds the prefill kernels' consumer-side waits at
+    that many polls (0: they give up at once); a negative value restores the default."""
+    load_library().kda_testing_set_wait_limit(int(polls))
 
 
 def _dtype_code(t: torch.Tensor, what: str) -> int:

@@ -126,8 +126,8 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
  *   - Limit: a call that runs on the tensor cores (bf16 q/k/v, dk = dv = 128, T_total > 0) and whose
  *     kda_chunk_fwd_workspace_size(...) exceeds KDA_STATIC_SCRATCH_BYTES returns KDA_ERR_UNSUPPORTED
  *     before any CUDA call.  The size is one 160.5 KB chunk record per 64-token chunk slot and head
- *     (slots = T_total / 64 + N + 1) plus 128 KB per (sequence, head); e.g. 2 sequences x 2048
- *     tokens x 2 heads need 21.5 MiB.  Every other call (fp32 q/k/v, dk or dv = 64) reads no scratch
+ *     (slots = T_total / 64 + N + 1) plus 128 KB per (sequence, head) and 4 bytes per sequence; e.g. 2
+ *     sequences x 2048 tokens x 2 heads need 21.5 MiB.  Every other call (fp32 q/k/v, dk or dv = 64) reads no scratch
  *     and has no limit, whatever kda_chunk_fwd_workspace_size says for its sizes.
  *   - Nothing in the scratch has to start at zero: every part a call reads is written earlier in the
  *     same call.

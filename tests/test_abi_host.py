@@ -26,6 +26,13 @@ def test_every_declared_symbol_is_exported(lib):
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
 
 
+def test_wait_limit_hook_needs_no_device(lib):
+    # the test hook only sets a process-wide number; restore the default afterwards
+    kda.kda_testing_set_wait_limit(0)
+    kda.kda_testing_set_wait_limit(-1)
+    assert "kda_testing_set_wait_limit" in kda.header_symbols()
+
+
 def test_status_strings_and_version(lib):
     assert kda.kda_status_string(kda.KDA_OK) == "ok"
     for st in range(1, 6):
@@ -126,9 +133,10 @@ def test_workspace_size_is_a_pure_host_function(lib):
     assert lib.kda_chunk_fwd_workspace_size(-1, 1, 1, 128, 128, 64) == 0
     assert kda.kda_chunk_fwd_workspace_size(4096, 1, 1, 64, 64) == 0   # the fp32 / d=64 paths use none
     # one 160.5 KB record per (chunk slot, head), slots = T / 64 + N + 1; then two fp32 128 x 128 states
-    # per (sequence, head) for the scan's intra-sequence split
-    assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) == (512 + 2) * 32 * 164352 + 2 * 32 * 65536
-    assert kda.kda_chunk_fwd_workspace_size(1000, 3, 2, 128, 128) == (15 + 4) * 2 * 164352 + 2 * 6 * 65536
+    # per (sequence, head) for the scan's intra-sequence split and the scan's sequence order (int32 [N],
+    # padded to 16 bytes)
+    assert kda.kda_chunk_fwd_workspace_size(32768, 1, 32, 128, 128) == (512 + 2) * 32 * 164352 + 2 * 32 * 65536 + 16
+    assert kda.kda_chunk_fwd_workspace_size(1000, 3, 2, 128, 128) == (15 + 4) * 2 * 164352 + 2 * 6 * 65536 + 16
 
 
 def test_static_scratch_rejects_oversize_before_any_cuda_call(lib):

@@ -72,5 +72,6 @@ def test_record_size_matches_the_workspace_size(wy):
     kbuild.build()
     kda.load_library()
     T, N, H = 5000, 3, 4
+    # the records, then the scan's two fp32 state arrays and its longest-first order (int32 [N], padded to 16 B)
     assert kda.kda_chunk_fwd_workspace_size(T, N, H, 128, 128) == \
-        wy.num_slots(T, N) * H * wy.rec_bytes() + 2 * N * H * 128 * 128 * 4
+        wy.num_slots(T, N) * H * wy.rec_bytes() + 2 * N * H * 128 * 128 * 4 + 16
