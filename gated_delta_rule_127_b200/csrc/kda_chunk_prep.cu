@@ -97,14 +97,19 @@ constexpr uint32_t OFF_SV0 = OFF_KP + 24576;
 constexpr uint32_t OFF_SV1 = OFF_KP + 57344;
 constexpr uint32_t OFF_MISC = 212992;  // beta[2][64] (this task, the next), e^{g_C} [128], strong-decay channel
                                        //   masks [4 blocks][4 words]
-constexpr uint32_t MISC_BYTES = (128 + 128) * 4 + 64;
+constexpr uint32_t MISC_BYTES = (128 + 128) * 4 + 64 + 16;  // ... and the wide-chunk flag
 constexpr uint32_t OFF_TASK = OFF_MISC + MISC_BYTES;  // three Task slots (this task, the next, the one after)
-constexpr uint32_t OFF_BARS = OFF_TASK + 96;   // mbarriers: TMA, MMA 1, MMA 2, MMA 3, MMA 4; then the TMEM base
-constexpr uint32_t OFF_SAL = OFF_BARS + 48;    // scalar log-decay [2][64] (Gated DeltaNet gates), by task parity
+constexpr uint32_t OFF_BARS = OFF_TASK + 96;   // mbarriers: TMA, MMA 1, MMA 2, MMA 3, MMA 4, v; then the TMEM base
+constexpr uint32_t OFF_SAL = OFF_BARS + 64;    // scalar log-decay [2][64] (Gated DeltaNet gates), by task parity
 constexpr uint32_t OFF_RN = OFF_SAL + 512;     // 1 / ||k_r|| [64], 1 / ||q_r|| [64] (fused L2 normalisation)
 constexpr uint32_t SMEM_USED = OFF_RN + 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
-// after MMA 1 (the column tiles are dead):
+// one-anchor chunks (every channel's log-decay spans at most kSpanLimit over the chunk): the MMA 1
+// operands in shared memory, over the log-decay staging and the column tiles
+constexpr uint32_t OFF_XF = OFF_G;             // [K; Q] e^{G - a} K-major rows n (128) x K c (128), sw128_off(n, c, 128)
+constexpr uint32_t OFF_YF = OFF_G + 65536;     // K e^{a - G} K-major rows i (64) x K c (128), sw128_off(i, c, 64)
+static_assert(OFF_YF + 32768 <= OFF_KP && OFF_YF % 1024 == 0, "one-anchor operands");
+// after MMA 1 (its operands are dead):
 constexpr uint32_t OFF_A = OFF_Y;              // A fp32 [64][TP]
 constexpr uint32_t OFF_T32 = OFF_Y + 17408;    // T fp32 [64][TP]
 constexpr uint32_t OFF_TIMG = OFF_Y + 35840;   // T K-major rows r x K s (64), B of MMA 2
@@ -367,6 +372,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float* s_beta2 = reinterpret_cast<float*>(sm + OFF_MISC);  // [2][64], by task parity
     float* s_gam = s_beta2 + 128;   // [128] e^{g_C}
     uint32_t* s_strong = reinterpret_cast<uint32_t*>(s_gam + 128);  // [4 blocks][4 words] strong-decay channels
+    volatile uint32_t* s_wide = s_strong + 16;  // set when some channel's log-decay spans more than kSpanLimit
     float* x_part = reinterpret_cast<float*>(sm + OFF_XP);     // [16 groups][128]
     float* f_anc = reinterpret_cast<float*>(sm + OFF_FAC);     // [4][128] anchors
     float* f_tau = f_anc + 512;     // [4][128] e^{g_e - a}
@@ -382,19 +388,21 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t* bar_m2 = bar_tma + 2;
     uint64_t* bar_m3 = bar_tma + 3;
     uint64_t* bar_m4 = bar_tma + 4;
-    uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 40);
+    uint64_t* bar_v = bar_tma + 5;
+    uint32_t* slot_tm = reinterpret_cast<uint32_t*>(sm + OFF_BARS + 48);
 
     constexpr uint32_t kGateBytes = SG ? 0 : C * DK * sizeof(TG);
-    constexpr uint32_t kStageBytes = 3 * C * DK * 2 + kGateBytes;
-    // Tile j (k, q, v, log_alpha) of a task into the staging buffers: one box covering all of the
-    // tile's 128-byte column blocks (completion on bar_tma, whose expected byte count kStageBytes is
-    // set once per task).  The four are issued by different warps.
-    // Boxes 0..2: k, q, log_alpha (issued by warps 0..2, SG: k, q); boxes 3, 4: the two 64-channel halves
-    // of v (into the P_lo rows of [Kt; P], so the next task's v is loaded only once MMAs 3 and 4 are done)
+    constexpr uint32_t kStageBytes = 2 * C * DK * 2 + kGateBytes;
+    constexpr uint32_t kVBytes = C * DV * 2;
+    // Tile j of a task into its staging buffer, one box covering all of the tile's 128-byte column
+    // blocks.  Boxes 0..2: k, q, log_alpha (SG: k, q), issued by warps 0..2, completing on bar_tma (its
+    // expected byte count kStageBytes set once per task).  Boxes 3, 4: the two 64-channel halves of v, in
+    // the P_lo rows of [Kt; P]: the next task's v is loaded once MMAs 3 and 4 are done, and completes on
+    // bar_v, which is awaited only by the pass that reads v.
     constexpr int kLoads = SG ? 2 : 3;
     auto load_box = [&](const Task& t, int j) {
         if (j >= 3) {
-            tma_load_4d(sm + (j == 3 ? OFF_SV0 : OFF_SV1), &tm_v, 0, static_cast<int>(t.c0), j - 3, t.h, bar_tma);
+            tma_load_4d(sm + (j == 3 ? OFF_SV0 : OFF_SV1), &tm_v, 0, static_cast<int>(t.c0), j - 3, t.h, bar_v);
             return;
         }
         const CUtensorMap* m = j == 0 ? &tm_k : j == 1 ? &tm_q : &tm_g;
@@ -403,7 +411,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     };
 
     uint32_t loads_issued = 0;    // thread 0: staging loads issued (bar_tma phases)
-    bool v_pending = false;       // thread 0: the last phase's v boxes are not issued yet
+    uint32_t v_issued = 0;        // thread 0: v loads issued (bar_v phases)
     TaskWalker walker;            // the last thread's: it looks the tasks up
     constexpr int kWalker = THREADS - 1;
     if (tid == kWalker) {
@@ -413,7 +421,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         slots[2].id = -1;
     }
     if (tid == 0) {
-        for (int b = 0; b < 5; ++b) mbar_init(bar_tma + b, 1);
+        for (int b = 0; b < 6; ++b) mbar_init(bar_tma + b, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
         if (!SG) tma_prefetch_desc(&tm_g);
@@ -423,9 +431,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0 && slots[0].id >= 0) {
         mbar_arrive_expect_tx(bar_tma, kStageBytes);
         for (int j = 0; j < kLoads; ++j) load_box(slots[0], j);
+        ++loads_issued;
+        mbar_arrive_expect_tx(bar_v, kVBytes);
         load_box(slots[0], 3);
         load_box(slots[0], 4);
-        ++loads_issued;
+        ++v_issued;
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -519,6 +529,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             x_part[(4 * I + qr) * 128 + c] = run;
         }
+        if (tid == 0) *s_wide = 0u;  // (read only after the barrier that ends step 2)
         float a_first[4];  // log-decay of each block's first row (the thread with rbq = 0 holds it as g[I][0])
 #pragma unroll
         for (int I = 0; I < 4; ++I) a_first[I] = a_at(16 * I, swf0, swb0);
@@ -540,6 +551,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         //      channel c (the four threads of a channel compute the same; those with qr = 0 publish them)
         float anc[4], gl[4];
         uint32_t strong = 0;  // bit I: block I's span exceeds kSpanLimit
+        float a_one;          // the chunk's one anchor for channel c (midpoint of its log-decay span)
         {
             float off = 0.f;
             float gfst[4];
@@ -561,6 +573,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 strong |= st ? (1u << I) : 0u;
                 anc[I] = st ? gfst[I] : gfst[I] - 0.5f * span;
             }
+            const float span_all = gfst[0] - gl[3];
+            if (span_all > kSpanLimit) *s_wide = 1u;
+            a_one = gfst[0] - 0.5f * span_all;
             // block I = qr's factors for channel c (the four threads of the channel split the blocks)
 #pragma unroll
             for (int I = 0; I < 4; ++I) {
@@ -576,8 +591,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (I == 3) s_gam[c] = __expf(gl[3]);
             }
         }
-        if (tid == 0) bulk_wait_read();  // the previous record's [Mt; Qh] tile has left shared memory
+        // v (awaited here, late, as it is loaded last) and the previous record's [Mt; Qh] tile out of
+        // shared memory; a timed-out wait is acted on at MMA 1's
+        const bool vlate = !mbar_wait(bar_v, par, wait_polls);
+        if (tid == 0) bulk_wait_read();
         const bool any_strong = __syncthreads_or(strong != 0);
+        // one anchor per channel for the whole chunk when no channel's log-decay spans more than
+        // kSpanLimit over it (every factor is then <= e^{kSpanLimit / 2}); else four 16-row blocks
+        const bool one = *s_wide == 0u;
 
         // ---- 3: per element (row i, channel c): the row factor e^{g_i - a} (for the row pass; g itself when
         //      some channel decays strongly), the column tiles of MMA 1, Kt^T (MMAs 3-4), (beta K e^G)^T,
@@ -635,13 +656,60 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tmem_st4(tq + TM_QG + 16 * I + rbq, qg);
             }
         };
-        if (len == C) elementwise(std::true_type{});
-        else elementwise(std::false_type{});
-        __syncthreads();
+        // one anchor: per element the factor e^{a - g_i} (<= e^{kSpanLimit / 2} either way) and its
+        // reciprocal give both MMA 1 operands straight from the element: rows i and 64 + i of
+        // X = [K; Q] e^{G - a}, row i of Y = K e^{a - G}; then Kt^T = (K e^{a - G})^T e^{g_C - a},
+        // (beta K e^G)^T, (beta V)^T and (Q e^G)^T as in the four-block pass (e^{g_i} = e^{g_i - a} e^{a})
+        auto elementwise_one = [&](auto full_chunk) {
+            constexpr bool kFull = decltype(full_chunk)::value;
+            const float kap = __expf(gl[3] - a_one), ea = __expf(a_one);
+            unsigned char* xcol = sm + OFF_XF + q4 * 16384;  // K-block of channel c
+            unsigned char* ycol = sm + OFF_YF + q4 * 8192;
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+                float kt[4], bk[4], bv[4], qg[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const int i = 16 * I + rbq + w;
+                    const bool live = kFull || i < len;
+                    const uint32_t ob = swb[w] + i * 128;
+                    float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK + ob));
+                    float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ + ob));
+                    float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + vbox + (ob - vblk)));
+                    if (PRO) { kv *= s_rn[i]; qv *= s_rn[64 + i]; }
+                    if (!live) { kv = 0.f; qv = 0.f; vv = 0.f; }
+                    const float b = s_beta[i];
+                    const float dc = __expf(a_one - g[I][w]);  // e^{a - g_i}
+                    const float rowf = recip_approx(dc);       // e^{g_i - a}
+                    const uint32_t o = swf[w] + i * 128;
+                    const float ky = kv * dc;
+                    *reinterpret_cast<float*>(ycol + o) = to_tf32(ky);
+                    *reinterpret_cast<float*>(xcol + o) = to_tf32(kv * rowf);
+                    *reinterpret_cast<float*>(xcol + 8192 + o) = to_tf32(qv * rowf);  // row 64 + i
+                    const float Gm = rowf * ea;
+                    kt[w] = to_tf32(ky * kap);
+                    bk[w] = to_tf32(b * kv * Gm);
+                    bv[w] = to_tf32(b * vv);
+                    qg[w] = qv * Gm;
+                }
+                *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+                tmem_st4(tq + TM_BK + 16 * I + rbq, bk);
+                tmem_st4(tq + TM_BV + 16 * I + rbq, bv);
+                tmem_st4(tq + TM_QG + 16 * I + rbq, qg);
+            }
+        };
+        if (one) {
+            if (len == C) elementwise_one(std::true_type{});
+            else elementwise_one(std::false_type{});
+        } else {
+            if (len == C) elementwise(std::true_type{});
+            else elementwise(std::false_type{});
+            __syncthreads();
+        }
 
         // ---- row pass: X = [K; Q] e^{G - a} into tensor memory (lane = row: 0..63 K, 64..127 Q; a the anchor
         //      of the row's block), channels 32 qr ..
-        {
+        if (!one) {
             const bool isq = c >= 64;
             const int r = c & 63, R = r >> 4;
             const unsigned char* src = sm + (isq ? OFF_SQ : OFF_SK);
@@ -678,24 +746,60 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_before_sync();
         __syncthreads();
 
-        // ---- MMA 1: [A_raw; P] = X Y^T (M=128, N=160, K=128): row r of block R uses the columns of tile R
+        // ---- MMA 1: [A_raw; P] = X Y^T (M=128, K=128).  Four blocks: N=160, X in tensor memory, row r of
+        //      block R uses the columns of tile R; one anchor: N=64, both operands in shared memory
         if (tid == 0) {
             tc_fence_after_sync();
-            const uint64_t by = sw128_desc(sbase + OFF_Y, 16, 1024);
-            constexpr uint32_t id1 = idesc_tf32(128, 160, false, false);
+            if (one) {
+                const uint64_t ax = sw128_desc(sbase + OFF_XF, 16, 1024);
+                const uint64_t by = sw128_desc(sbase + OFF_YF, 16, 1024);
+                constexpr uint32_t id1 = idesc_tf32(128, 64, false, false);
 #pragma unroll
-            for (int kk = 0; kk < DK / 8; ++kk)
-                mma_tf32_ts(tmem + TM_D1, tmem + TM_X + 8 * kk, by + (((kk >> 2) * 160 * 128 + (kk & 3) * 32) >> 4), id1,
-                            kk > 0);
+                for (int kk = 0; kk < DK / 8; ++kk)
+                    mma_tf32(tmem + TM_D1, ax + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                             by + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id1, kk > 0);
+            } else {
+                const uint64_t by = sw128_desc(sbase + OFF_Y, 16, 1024);
+                constexpr uint32_t id1 = idesc_tf32(128, 160, false, false);
+#pragma unroll
+                for (int kk = 0; kk < DK / 8; ++kk)
+                    mma_tf32_ts(tmem + TM_D1, tmem + TM_X + 8 * kk, by + (((kk >> 2) * 160 * 128 + (kk & 3) * 32) >> 4),
+                                id1, kk > 0);
+            }
             mma_commit(bar_m1);
             mma_issued |= 1u;
         }
-        failed = !mbar_wait(bar_m1, par, wait_polls);
+        failed = !mbar_wait(bar_m1, par, wait_polls) || vlate;
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        {   // lane rows 0..63 -> A (beta-scaled, strictly lower, fp32); 64..127 -> P (lower with the
-            // diagonal).  Lanes 0-15 of the warp are rows of block R0, lanes 16-31 of block R0 + 1; the
-            // warp reads its blocks' columns in 16-column pieces, the four warps of a quadrant in turn.
+        if (one) {  // lane rows 0..63 -> A (beta-scaled, strictly lower, fp32); 64..127 -> P (lower with the
+                    // diagonal); columns 16 qr ..
+            const bool isq = c >= 64;
+            const int row = c & 63, i0 = 16 * qr;
+            float x[16];
+            tmem_ld16(tq + TM_D1 + i0, x);
+            if (!isq) {
+                const float b = s_beta[row];
+                float* arow = reinterpret_cast<float*>(sm + OFF_A) + row * TP + i0;
+#pragma unroll
+                for (int k4 = 0; k4 < 16; k4 += 4) {
+                    float a[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) a[u] = (i0 + k4 + u) < row ? b * x[k4 + u] : 0.f;
+                    *reinterpret_cast<float4*>(arow + k4) = make_float4(a[0], a[1], a[2], a[3]);
+                }
+            } else {
+#pragma unroll
+                for (int k4 = 0; k4 < 16; k4 += 4) {
+                    float p[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) p[u] = (i0 + k4 + u) <= row ? x[k4 + u] : 0.f;
+                    put_p(row, i0 + k4, p);
+                }
+            }
+        } else {  // lane rows 0..63 -> A, 64..127 -> P as above.  Lanes 0-15 of the warp are rows of block
+                  // R0, lanes 16-31 of block R0 + 1; the warp reads its blocks' columns in 16-column pieces,
+                  // the four warps of a quadrant in turn.
             const bool isq = c >= 64;
             const int row = c & 63, Rl = row >> 4;
             const int R0 = 2 * (q4 & 1), n0 = R0 + 1, ntot = 2 * R0 + 3;
@@ -792,7 +896,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (tid == 0 && tn.id >= 0) {
             mbar_arrive_expect_tx(bar_tma, kStageBytes);
             ++loads_issued;
-            v_pending = true;  // v once MMAs 3 and 4 have read the P_lo rows it lands in
         }
         __syncthreads();
         if (lane == 0 && warp < kLoads && tn.id >= 0) load_box(tn, warp);
@@ -948,10 +1051,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_before_sync();
         if (__syncthreads_or(late)) { failed = true; break; }
         if (tid == 0) {
-            if (v_pending) {
+            if (tn.id >= 0) {  // v once MMAs 3 and 4 have read the P_lo rows it lands in
+                mbar_arrive_expect_tx(bar_v, kVBytes);
                 load_box(tn, 3);
                 load_box(tn, 4);
-                v_pending = false;
+                ++v_issued;
             }
             bulk_store(rec + wy::REC_MQ, sm + OFF_STG, wy::REC_MQ_BYTES);
             bulk_commit();
@@ -964,11 +1068,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // that was committed
         for (int k = 0; k < 4; ++k)
             if (mma_issued & (1u << k)) mbar_wait(bar_m1 + k, cur_par, kWaitPolls);
-        if (v_pending) {  // complete the pending phase (its other boxes are in flight), now that no MMA reads P_lo
-            load_box(slots[cur == 2 ? 0 : cur + 1], 3);
-            load_box(slots[cur == 2 ? 0 : cur + 1], 4);
-        }
         if (loads_issued > 0) mbar_wait(bar_tma, (loads_issued - 1) & 1, kWaitPolls);
+        if (v_issued > 0) mbar_wait(bar_v, (v_issued - 1) & 1, kWaitPolls);
         raise_flag(flags, KDA_DEVFLAG_TIMEOUT);
     }
     if (tid == 0) bulk_wait_read();  // the bulk copies read shared memory until they complete
