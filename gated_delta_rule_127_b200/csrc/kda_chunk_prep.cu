@@ -102,7 +102,8 @@ constexpr uint32_t OFF_TASK = OFF_MISC + MISC_BYTES;  // three Task slots (this 
 constexpr uint32_t OFF_BARS = OFF_TASK + 96;   // mbarriers: TMA, MMA 1, MMA 2, MMA 3, MMA 4, v; then the TMEM base
 constexpr uint32_t OFF_SAL = OFF_BARS + 64;    // scalar log-decay [2][64] (Gated DeltaNet gates), by task parity
 constexpr uint32_t OFF_RN = OFF_SAL + 512;     // 1 / ||k_r|| [64], 1 / ||q_r|| [64] (fused L2 normalisation)
-constexpr uint32_t SMEM_USED = OFF_RN + 512;
+constexpr uint32_t OFF_WALK = OFF_RN + 512;   // the task walker's state (one thread's; kept out of registers)
+constexpr uint32_t SMEM_USED = OFF_WALK + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base to 1024
 // one-anchor chunks (every channel's log-decay spans at most kSpanLimit over the chunk): the MMA 1
 // operands in shared memory, over the log-decay staging and the column tiles
@@ -253,7 +254,8 @@ struct TaskWalker {
 };
 
 // One 16 x 8 tile of X Y on the warp's tensor cores (mma.sync m16n8k8, tf32 operands rounded to
-// nearest, fp32 accumulation): X row-major with row stride xs (the tile's 16 rows, K = kn columns), Y
+// nearest by to_tf32_op, fp32 accumulation): X row-major with row stride xs (the tile's 16 rows, K = kn
+// columns), Y
 // row-major with row stride ys (K = kn rows, the tile's 8 columns).  Fragment layout of the m16n8k8
 // tf32 shape: lane = 4 g + t holds X[g][t], X[g+8][t], X[g][t+4], X[g+8][t+4] and Y[t][g], Y[t+4][g],
 // and receives D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1].
@@ -261,12 +263,12 @@ __device__ __forceinline__ void warp_tile_16x8(const float* x, int xs, const flo
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     d[0] = d[1] = d[2] = d[3] = 0.f;
     for (int k0 = 0; k0 < kn; k0 += 8) {
-        const uint32_t a0 = __float_as_uint(to_tf32(x[g * xs + k0 + t]));
-        const uint32_t a1 = __float_as_uint(to_tf32(x[(g + 8) * xs + k0 + t]));
-        const uint32_t a2 = __float_as_uint(to_tf32(x[g * xs + k0 + t + 4]));
-        const uint32_t a3 = __float_as_uint(to_tf32(x[(g + 8) * xs + k0 + t + 4]));
-        const uint32_t b0 = __float_as_uint(to_tf32(y[(k0 + t) * ys + g]));
-        const uint32_t b1 = __float_as_uint(to_tf32(y[(k0 + t + 4) * ys + g]));
+        const uint32_t a0 = __float_as_uint(to_tf32_op(x[g * xs + k0 + t]));
+        const uint32_t a1 = __float_as_uint(to_tf32_op(x[(g + 8) * xs + k0 + t]));
+        const uint32_t a2 = __float_as_uint(to_tf32_op(x[g * xs + k0 + t + 4]));
+        const uint32_t a3 = __float_as_uint(to_tf32_op(x[(g + 8) * xs + k0 + t + 4]));
+        const uint32_t b0 = __float_as_uint(to_tf32_op(y[(k0 + t) * ys + g]));
+        const uint32_t b1 = __float_as_uint(to_tf32_op(y[(k0 + t + 4) * ys + g]));
         asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
                      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -282,74 +284,79 @@ __device__ __forceinline__ void warp_store_16x8(float* z, int zs, const float (&
     z[(g + 8) * zs + 2 * t + 1] = sg * d[3];
 }
 
-// T = (I + A)^{-1} for A strictly lower (fp32, row stride TP) into tm, fully written (zero above the
-// diagonal).  xs: 1024 floats of scratch.  The 16 x 16 diagonal blocks by forward substitution in fp32,
-// then two merges of [[T1, 0], [T21, T2]] with T21 = -T2 A21 T1: 16 -> 32 (both halves at once) and
-// 32 -> 64, whose products run as 16 x 8 tiles on the warps' tensor cores with tf32 operands (these
-// blocks reach the rest of the chunk only through tf32 products; an fp64 emulation against the
-// oracle shows no loss from it).
-__device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, float* xs) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (warp < 4) {
-        if (lane < 16) {  // warp w inverts diagonal block w, lane j solves for column j
-            const int b = 16 * warp, j = lane;
-            float t[16];
+// T = (I + A)^{-1} for A strictly lower (fp32, row stride TP) into tm, the part on and below the
+// diagonal blocks (zero_above_blocks writes the rest); xs: 1024 floats of scratch.  Run by four warps,
+// iw = 0..3 their index, joined by named barrier 1.  The 16 x 16 diagonal blocks by forward
+// substitution in fp32, then two merges of [[T1, 0], [T21, T2]] with T21 = -T2 (A21 T1): 16 -> 32 (both
+// halves at once) and 32 -> 64.  Their products run as 16 x 8 tiles on the warps' tensor cores with tf32
+// operands (these blocks reach the rest of the chunk only through tf32 products; an fp64 emulation
+// against the oracle shows no loss from it).  In each merge warp iw owns one 8-column strip of T21,
+// whose two products need only that strip of A21 T1: the warp forms it, passes it through its own
+// scratch and goes on.  No product reads the zeros above the diagonal blocks.
+__device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, float* xs, int iw) {
+    const int lane = threadIdx.x & 31;
+    if (lane < 16) {  // warp iw inverts diagonal block iw, lane j solves for column j
+        const int b = 16 * iw, j = lane;
+        float t[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float a[16];  // row r of the block (columns < r are used), broadcast reads
+        for (int r = 0; r < 16; ++r) {
+            float a[16];  // row r of the block (columns < r are used), broadcast reads
 #pragma unroll
-                for (int i4 = 0; i4 < 16; i4 += 4) {
-                    if (i4 < r) {
-                        const float4 v = *reinterpret_cast<const float4*>(am + (b + r) * TP + b + i4);
-                        a[i4] = v.x; a[i4 + 1] = v.y; a[i4 + 2] = v.z; a[i4 + 3] = v.w;
-                    }
+            for (int i4 = 0; i4 < 16; i4 += 4) {
+                if (i4 < r) {
+                    const float4 v = *reinterpret_cast<const float4*>(am + (b + r) * TP + b + i4);
+                    a[i4] = v.x; a[i4 + 1] = v.y; a[i4 + 2] = v.z; a[i4 + 3] = v.w;
                 }
-                float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-                for (int i = 0; i < r; ++i) {
-                    if (i & 1) acc1 -= a[i] * t[i];
-                    else acc0 -= a[i] * t[i];
-                }
-                t[r] = (r >= j) ? acc0 + acc1 : 0.f;
             }
+            float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) tm[(b + r) * TP + b + j] = t[r];
+            for (int i = 0; i < r; ++i) {
+                if (i & 1) acc1 -= a[i] * t[i];
+                else acc0 -= a[i] * t[i];
+            }
+            t[r] = (r >= j) ? acc0 + acc1 : 0.f;
         }
-    } else {  // zeros above the diagonal blocks: rows r, columns 16 (r / 16 + 1) .. 63
-        for (int e = tid - 128; e < 64 * 64; e += THREADS - 128) {
-            const int r = e >> 6, col = e & 63;
-            if (col >= 16 * ((r >> 4) + 1)) tm[r * TP + col] = 0.f;
-        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) tm[(b + r) * TP + b + j] = t[r];
     }
-    __syncthreads();
-    const int p = warp >> 1, nt = warp & 1;  // 16 -> 32: warps 0..3, block pair p, 8-column tile nt
-    if (warp < 4) {  // X_p = A_{2p+1,2p} T_{2p,2p}
-        float d[4];
+    group_sync(1, 128);
+    float d[4];
+    {   // 16 -> 32, block pair p, strip nt: X = A_{2p+1,2p} T_{2p,2p}[:, strip], then
+        // T_{2p+1,2p}[:, strip] = -T_{2p+1,2p+1} X
+        const int p = iw >> 1, nt = iw & 1;
+        float* xw = xs + iw * 128;  // 16 x 8, row stride 8
         warp_tile_16x8(am + (32 * p + 16) * TP + 32 * p, TP, tm + (32 * p) * TP + 32 * p + 8 * nt, TP, 16, d);
-        warp_store_16x8(xs + p * 256 + 8 * nt, 16, d, false);
-    }
-    __syncthreads();
-    if (warp < 4) {  // T_{2p+1,2p} = -T_{2p+1,2p+1} X_p
-        float d[4];
-        warp_tile_16x8(tm + (32 * p + 16) * TP + 32 * p + 16, TP, xs + p * 256 + 8 * nt, 16, 16, d);
+        warp_store_16x8(xw, 8, d, false);
+        __syncwarp();
+        warp_tile_16x8(tm + (32 * p + 16) * TP + 32 * p + 16, TP, xw, 8, 16, d);
         warp_store_16x8(tm + (32 * p + 16) * TP + 32 * p + 8 * nt, TP, d, true);
     }
-    __syncthreads();
-    const int mt = warp >> 2, ct = warp & 3;  // 32 -> 64: warps 0..7, 16-row tile mt, 8-column tile ct
-    if (warp < 8) {  // X = A21 T1
-        float d[4];
-        warp_tile_16x8(am + (32 + 16 * mt) * TP, TP, tm + 8 * ct, TP, 32, d);
-        warp_store_16x8(xs + (16 * mt) * 32 + 8 * ct, 32, d, false);
+    group_sync(1, 128);
+    {   // 32 -> 64, strip ct: X = A21 T1[:, strip] (T1's strips 2, 3 are zero above row 16), then
+        // T21[:, strip] = -T2 X (T2's rows 0..15 are zero right of column 16)
+        const int ct = iw, k0 = ct < 2 ? 0 : 16;
+        float* xw = xs + iw * 256;  // 32 x 8, row stride 8
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            warp_tile_16x8(am + (32 + 16 * mt) * TP + k0, TP, tm + k0 * TP + 8 * ct, TP, 32 - k0, d);
+            warp_store_16x8(xw + 128 * mt, 8, d, false);
+        }
+        __syncwarp();
+        warp_tile_16x8(tm + 32 * TP + 32, TP, xw, 8, 16, d);
+        warp_store_16x8(tm + 32 * TP + 8 * ct, TP, d, true);
+        warp_tile_16x8(tm + 48 * TP + 32, TP, xw, 8, 32, d);
+        warp_store_16x8(tm + 48 * TP + 8 * ct, TP, d, true);
     }
-    __syncthreads();
-    if (warp < 8) {  // T21 = -T2 X
-        float d[4];
-        warp_tile_16x8(tm + (32 + 16 * mt) * TP + 32, TP, xs + 8 * ct, 32, 32, d);
-        warp_store_16x8(tm + (32 + 16 * mt) * TP + 8 * ct, TP, d, true);
-    }
-    __syncthreads();
 }
-
+// The zeros of T above its diagonal blocks (rows r, columns 16 (r / 16 + 1) .. 63), by 128 threads
+// (t = 0..127), four at a time.
+__device__ __forceinline__ void zero_above_blocks(float* tm, int t) {
+#pragma unroll
+    for (int e = t; e < 64 * 16; e += 128) {
+        const int r = e >> 4, c4 = (e & 15) * 4;
+        if (c4 >= 16 * ((r >> 4) + 1)) *reinterpret_cast<float4*>(tm + r * TP + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
 
 // SG: Gated DeltaNet gates -- log_alpha is [T_total, H], one decay rate per token and head, read
 // with beta and broadcast over the key channels (tm_g is then unused).
@@ -412,12 +419,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     uint32_t loads_issued = 0;    // thread 0: staging loads issued (bar_tma phases)
     uint32_t v_issued = 0;        // thread 0: v loads issued (bar_v phases)
-    TaskWalker walker;            // the last thread's: it looks the tasks up
+    // the last thread looks the tasks up; its walker lives in shared memory, so that no thread holds
+    // the walker's state in registers through the task loop
+    TaskWalker* walker = reinterpret_cast<TaskWalker*>(sm + OFF_WALK);
+    static_assert(sizeof(TaskWalker) <= 128, "walker state");
     constexpr int kWalker = THREADS - 1;
     if (tid == kWalker) {
-        walker.init(cu_seqlens, T_total, N, H, ws, flags);
-        slots[0] = walker.next();
-        slots[1] = walker.next();
+        walker->init(cu_seqlens, T_total, N, H, ws, flags);
+        slots[0] = walker->next();
+        slots[1] = walker->next();
         slots[2].id = -1;
     }
     if (tid == 0) {
@@ -467,7 +477,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             hi[u] = to_tf32(p[u]);
-            lo[u] = to_tf32(p[u] - hi[u]);
+            lo[u] = to_tf32_op(p[u] - hi[u]);
         }
         *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(128 + t, i, 256)) = make_float4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(192 + t, i, 256)) = make_float4(lo[0], lo[1], lo[2], lo[3]);
@@ -642,12 +652,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     // column tiles: (n, c) at q4 * 160 * 128 + n * 128 + swizzle, n = y_row(R) + i = i mod 8
                     unsigned char* ycol = sm + OFF_Y + q4 * 20480 + swf[w] + i * 128;
                     const float kf = kv * F;
-                    *reinterpret_cast<float*>(ycol + y_row(I) * 128) = to_tf32(kv * dc);
+                    *reinterpret_cast<float*>(ycol + y_row(I) * 128) = to_tf32_op(kv * dc);
 #pragma unroll
-                    for (int R = I + 1; R < 4; ++R) *reinterpret_cast<float*>(ycol + y_row(R) * 128) = to_tf32(kf * rho[R]);
-                    kt[w] = to_tf32(kf * kap);
-                    bk[w] = to_tf32(b * kv * Gm);
-                    bv[w] = to_tf32(b * vv);
+                    for (int R = I + 1; R < 4; ++R) *reinterpret_cast<float*>(ycol + y_row(R) * 128) = to_tf32_op(kf * rho[R]);
+                    kt[w] = to_tf32_op(kf * kap);
+                    bk[w] = to_tf32_op(b * kv * Gm);
+                    bv[w] = to_tf32_op(b * vv);
                     qg[w] = qv * Gm;
                 }
                 *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
@@ -683,13 +693,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const float rowf = recip_approx(dc);       // e^{g_i - a}
                     const uint32_t o = swf[w] + i * 128;
                     const float ky = kv * dc;
-                    *reinterpret_cast<float*>(ycol + o) = to_tf32(ky);
-                    *reinterpret_cast<float*>(xcol + o) = to_tf32(kv * rowf);
-                    *reinterpret_cast<float*>(xcol + 8192 + o) = to_tf32(qv * rowf);  // row 64 + i
+                    *reinterpret_cast<float*>(ycol + o) = to_tf32_op(ky);
+                    *reinterpret_cast<float*>(xcol + o) = to_tf32_op(kv * rowf);
+                    *reinterpret_cast<float*>(xcol + 8192 + o) = to_tf32_op(qv * rowf);  // row 64 + i
                     const float Gm = rowf * ea;
-                    kt[w] = to_tf32(ky * kap);
-                    bk[w] = to_tf32(b * kv * Gm);
-                    bv[w] = to_tf32(b * vv);
+                    kt[w] = to_tf32_op(ky * kap);
+                    bk[w] = to_tf32_op(b * kv * Gm);
+                    bv[w] = to_tf32_op(b * vv);
                     qg[w] = qv * Gm;
                 }
                 *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
@@ -733,7 +743,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int i = 0; i < 8; ++i) fv[i] = __expf(fv[i] - av[i]);
                 }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[8 * e8 + i] = to_tf32((PRO ? x[i] * rn : x[i]) * fv[i]);
+                for (int i = 0; i < 8; ++i) v[8 * e8 + i] = to_tf32_op((PRO ? x[i] * rn : x[i]) * fv[i]);
                 if (!live) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) v[8 * e8 + i] = 0.f;
@@ -772,13 +782,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         failed = !mbar_wait(bar_m1, par, wait_polls) || vlate;
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        if (one) {  // lane rows 0..63 -> A (beta-scaled, strictly lower, fp32); 64..127 -> P (lower with the
-                    // diagonal); columns 16 qr ..
+        if (one) {  // lane rows 0..63 -> A (beta-scaled, strictly lower, fp32), columns 16 qr ..; the P rows
+                    // are read during the inverse
             const bool isq = c >= 64;
             const int row = c & 63, i0 = 16 * qr;
-            float x[16];
-            tmem_ld16(tq + TM_D1 + i0, x);
             if (!isq) {
+                float x[16];
+                tmem_ld16(tq + TM_D1 + i0, x);
                 const float b = s_beta[row];
                 float* arow = reinterpret_cast<float*>(sm + OFF_A) + row * TP + i0;
 #pragma unroll
@@ -787,14 +797,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int u = 0; u < 4; ++u) a[u] = (i0 + k4 + u) < row ? b * x[k4 + u] : 0.f;
                     *reinterpret_cast<float4*>(arow + k4) = make_float4(a[0], a[1], a[2], a[3]);
-                }
-            } else {
-#pragma unroll
-                for (int k4 = 0; k4 < 16; k4 += 4) {
-                    float p[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) p[u] = (i0 + k4 + u) <= row ? x[k4 + u] : 0.f;
-                    put_p(row, i0 + k4, p);
                 }
             }
         } else {  // lane rows 0..63 -> A, 64..127 -> P as above.  Lanes 0-15 of the warp are rows of block
@@ -901,8 +903,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (lane == 0 && warp < kLoads && tn.id >= 0) load_box(tn, warp);
         load_beta(tn, par ^ 1u);
 
-        // ---- T = (I + A)^{-1}, then its tf32 operand tile
-        unit_lower_inverse(reinterpret_cast<const float*>(sm + OFF_A), reinterpret_cast<float*>(sm + OFF_T32), xs);
+        // ---- T = (I + A)^{-1} by warps 0, 1, 4, 5 (A-lane warps), the zeros above its diagonal blocks by
+        //      warps 8, 9, 12, 13; meanwhile, for one-anchor chunks, the P-lane warps move P into [Kt; P].
+        //      Then T's tf32 operand tile.
+        if (q4 < 2) {
+            if (warp < 8) unit_lower_inverse(reinterpret_cast<const float*>(sm + OFF_A), reinterpret_cast<float*>(sm + OFF_T32),
+                                             xs, (warp & 1) | ((warp >> 2) << 1));
+            else zero_above_blocks(reinterpret_cast<float*>(sm + OFF_T32), (tid & 31) | (((warp & 1) | (((warp >> 2) - 2) << 1)) << 5));
+        } else if (one) {  // lane rows 64..127: P (lower with the diagonal), columns 16 qr ..
+            const int row = c & 63, i0 = 16 * qr;
+            float x[16];
+            tmem_ld16(tq + TM_D1 + i0, x);
+#pragma unroll
+            for (int k4 = 0; k4 < 16; k4 += 4) {
+                float p[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) p[u] = (i0 + k4 + u) <= row ? x[k4 + u] : 0.f;
+                put_p(row, i0 + k4, p);
+            }
+        }
+        __syncthreads();
         {
             const float* t32 = reinterpret_cast<const float*>(sm + OFF_T32);
 #pragma unroll
@@ -911,7 +931,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int r = idx >> 4, s4 = (idx & 15) * 4;
                 const float4 t = *reinterpret_cast<const float4*>(t32 + r * TP + s4);
                 *reinterpret_cast<float4*>(sm + OFF_TIMG + sw128_off(r, s4, 64)) =
-                    make_float4(to_tf32(t.x), to_tf32(t.y), to_tf32(t.z), to_tf32(t.w));
+                    make_float4(to_tf32_op(t.x), to_tf32_op(t.y), to_tf32_op(t.z), to_tf32_op(t.w));
             }
         }
         fence_async_smem();
@@ -932,22 +952,25 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mma_commit(bar_m2);
             mma_issued |= 2u;
         }
-        if (tid == kWalker) slots[aft] = walker.next();  // while MMA 2 runs: the task after the next
+        if (tid == kWalker) slots[aft] = walker->next();  // while MMA 2 runs: the task after the next
         failed = !mbar_wait(bar_m2, par, wait_polls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        float qg[16];  // (Q e^G)^T of lane c, tokens 16 qr .. +15: moved into MMA 3's accumulator below
-        {   // -W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..)
-            float x[32];
+        uint32_t qg[16];  // (Q e^G)^T of lane c, tokens 16 qr .. +15: moved into MMA 3's accumulator below
+        {   // W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..)
+            uint32_t x[32];
             const bool isw = qr < 2;
-            tmem_ld32(tq + (isw ? TM_WT : TM_UT) + 32 * (qr & 1), x);
-            const float sgn = isw ? -1.f : 1.f;
+            tmem_ld32_nw(tq + (isw ? TM_WT : TM_UT) + 32 * (qr & 1), x);
+            tmem_ld16_nw(tq + TM_QG + 16 * qr, qg);
+            tmem_ld_wait();
+            after_ld_wait(x);
+            after_ld_wait(qg);
             unsigned char* tile = sm + (isw ? OFF_WT : OFF_UT);
+            auto r = [&](int e) { return to_tf32_op(__uint_as_float(x[e])); };
 #pragma unroll
             for (int e4 = 0; e4 < 32; e4 += 4)
                 *reinterpret_cast<float4*>(tile + sw128_off(c, 32 * (qr & 1) + e4, 128)) =
-                    make_float4(to_tf32(sgn * x[e4]), to_tf32(sgn * x[e4 + 1]), to_tf32(sgn * x[e4 + 2]), to_tf32(sgn * x[e4 + 3]));
-            tmem_ld16(tq + TM_QG + 16 * qr, qg);
+                    make_float4(r(e4), r(e4 + 1), r(e4 + 2), r(e4 + 3));
         }
         tc_fence_before_sync();
         __syncthreads();  // W^T, U^T and (Q e^G)^T are read: MMA 3's accumulator may be filled over them
@@ -958,7 +981,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
             for (int e = 0; e < 32; ++e) d[e] = (32 * qr + e == c) ? gam : 0.f;
             tmem_st32(tq + TM_DW + 32 * qr, d);
-            tmem_st16(tq + TM_DW + 128 + 16 * qr, qg);
+            float qf[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) qf[e] = __uint_as_float(qg[e]);
+            tmem_st16(tq + TM_DW + 128 + 16 * qr, qf);
             float z[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) z[e] = 0.f;
@@ -977,11 +1003,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint64_t aw = sw128_desc(sbase + OFF_WT, 16, 1024);
             const uint64_t au = sw128_desc(sbase + OFF_UT, 16, 1024);
             const uint64_t bkp = sw128_desc(sbase + OFF_KP, 16, 1024);
-            constexpr uint32_t id3 = idesc_tf32(128, 256, false, false);
+            constexpr uint32_t id4 = idesc_tf32(128, 256, false, false);
+            constexpr uint32_t id3 = idesc_tf32(128, 256, false, false, true);  // with -W^T
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)
                 mma_tf32(tmem + TM_DU, au + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                         bkp + (((kk >> 2) * 32768 + (kk & 3) * 32) >> 4), id3, kk > 0);
+                         bkp + (((kk >> 2) * 32768 + (kk & 3) * 32) >> 4), id4, kk > 0);
             mma_commit(bar_m4);
 #pragma unroll
             for (int kk = 0; kk < C / 8; ++kk)  // onto the seeded accumulator
@@ -995,8 +1022,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bool late = !mbar_wait(bar_m4, par, wait_polls);
         tc_fence_after_sync();
         {   // B^T (lane dv = c, rows i = 32 qr ..) and Uo^T (lane dv, tokens t = 16 qr ..) -> record
+            uint32_t xr[32], yh[16], yl[16];  // B^T; U^T P_hi^T and U^T P_lo^T
+            tmem_ld32_nw(tq + TM_DU + 32 * qr, xr);
+            tmem_ld16_nw(tq + TM_DU + 128 + 16 * qr, yh);
+            tmem_ld16_nw(tq + TM_DU + 192 + 16 * qr, yl);
+            tmem_ld_wait();
+            after_ld_wait(xr);
+            after_ld_wait(yh);
+            after_ld_wait(yl);
             float x[32];
-            tmem_ld32(tq + TM_DU + 32 * qr, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(xr[e]);
             float m = 0.f;
 #pragma unroll
             for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(x[e]));
@@ -1016,35 +1052,36 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 gb[(4 * qr + s8) * 128 + c] = make_uint4(w[0], w[1], w[2], w[3]);
             }
             reinterpret_cast<signed char*>(rec + wy::REC_BEXP)[qr * 128 + c] = static_cast<signed char>(ex);
-            float y[16], yl[16];  // U^T P_hi^T + U^T P_lo^T
-            tmem_ld16(tq + TM_DU + 128 + 16 * qr, y);
-            tmem_ld16(tq + TM_DU + 192 + 16 * qr, yl);
+            auto uo = [&](int e) { return __uint_as_float(yh[e]) + __uint_as_float(yl[e]); };
             float4* gu = reinterpret_cast<float4*>(rec + wy::REC_UO);
 #pragma unroll
             for (int s4 = 0; s4 < 4; ++s4)
-                gu[(4 * qr + s4) * 128 + c] = make_float4(y[4 * s4] + yl[4 * s4], y[4 * s4 + 1] + yl[4 * s4 + 1],
-                                                          y[4 * s4 + 2] + yl[4 * s4 + 2], y[4 * s4 + 3] + yl[4 * s4 + 3]);
+                gu[(4 * qr + s4) * 128 + c] = make_float4(uo(4 * s4), uo(4 * s4 + 1), uo(4 * s4 + 2), uo(4 * s4 + 3));
         }
         late |= !mbar_wait(bar_m3, par, wait_polls);
         tc_fence_after_sync();
         {   // Mt (lane j = c, rows i = 32 qr ..) and Qh (lane j, tokens t = 16 qr ..) into the record's [Mt; Qh]
             // tile in shared memory (for each row the warp's 32 lanes write one 128-byte run), then one bulk
             // copy.  The [Kt; P] and W^T, U^T tiles under it are dead: MMAs 3 and 4 are complete.
-            float x[32];
-            tmem_ld32(tq + TM_DW + 32 * qr, x);
+            uint32_t x[32], yh[16], yl[16];  // Mt^T; the hi and lo halves of Qh^T
+            tmem_ld32_nw(tq + TM_DW + 32 * qr, x);
+            tmem_ld16_nw(tq + TM_DW + 128 + 16 * qr, yh);
+            tmem_ld16_nw(tq + TM_DW + 192 + 16 * qr, yl);
+            tmem_ld_wait();
+            after_ld_wait(x);
+            after_ld_wait(yh);
+            after_ld_wait(yl);
             unsigned char* stg = sm + OFF_STG + q4 * wy::REC_MQ_KBLOCK + ((lane & 3) << 2);  // K-block of channel c
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const int i = 32 * qr + e;  // row i; its 16-byte chunks permuted by i % 8 = e % 8
-                *reinterpret_cast<float*>(stg + i * 128 + (((lane >> 2) ^ (e & 7)) << 4)) = to_tf32(x[e]);
+                *reinterpret_cast<float*>(stg + i * 128 + (((lane >> 2) ^ (e & 7)) << 4)) = to_tf32(__uint_as_float(x[e]));
             }
-            float y[16], sd[16];  // the hi and lo halves of Qh^T
-            tmem_ld16(tq + TM_DW + 128 + 16 * qr, y);
-            tmem_ld16(tq + TM_DW + 192 + 16 * qr, sd);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int n = 128 + 16 * qr + e;  // row of token t = 16 qr + e
-                *reinterpret_cast<float*>(stg + n * 128 + (((lane >> 2) ^ (e & 7)) << 4)) = to_tf32(y[e] + sd[e]);
+                *reinterpret_cast<float*>(stg + n * 128 + (((lane >> 2) ^ (e & 7)) << 4)) =
+                    to_tf32(__uint_as_float(yh[e]) + __uint_as_float(yl[e]));
             }
         }
         fence_async_smem();
