@@ -358,6 +358,86 @@ __device__ __forceinline__ void zero_above_blocks(float* tm, int t) {
     }
 }
 
+// ---- the four-block elementwise pass (chunks whose log-decay spans more than kSpanLimit over the
+// chunk for some channel).  Kept out of line: the kernel's registers are then allocated for the
+// one-anchor pass alone, and this pass's inputs are handed over in memory only when a chunk takes it.
+struct BlockPass {
+    float g[4][4];  // g of the thread's rows 16 I + 4 (w / 4) + w' (w = warp)
+    float anc[4], gl[4];
+    uint32_t swf[4], swb[4];
+    const float* s_beta;
+    uint32_t strong, tq, colf, vbox, vblk;
+    int len;
+    bool any_strong;
+};
+// Per element (row i, channel c): the row factor e^{g_i - a} (for the row pass; g itself when some
+// channel decays strongly), the column tiles of MMA 1, Kt^T (MMAs 3-4), (beta K e^G)^T, (beta V)^T
+// (MMA 2) and (Q e^G)^T.  For i in block I, F_i = e^{g_eI - g_i} <= 1 (eI the block's last row);
+// diagonal column factor e^{a_I - g_i} (1 / the row factor); column factor of a later block R:
+// e^{a_R - g_eI} F_i (both <= 1).
+template <bool PRO, bool kFull>
+__device__ __noinline__ void elementwise_blocks(const BlockPass& p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, qr = warp >> 2, rbq = 4 * qr, c = 32 * q4 + lane;
+    const float* f_tau = reinterpret_cast<const float*>(sm + OFF_FAC) + 512;
+    const float* f_kap = f_tau + 512;
+    const float* f_ea = f_kap + 512;
+    const float* f_rho = reinterpret_cast<const float*>(sm + OFF_RHO);
+    const float* s_rn = reinterpret_cast<const float*>(sm + OFF_RN);
+#pragma unroll
+    for (int I = 0; I < 4; ++I) {
+        const bool st = (p.strong >> I) & 1u;
+        const float tau = f_tau[I * 128 + c], kap = f_kap[I * 128 + c], ea = f_ea[I * 128 + c];
+        float rho[4];
+#pragma unroll
+        for (int R = I + 1; R < 4; ++R) rho[R] = f_rho[rho_idx(R, I) * 128 + c];
+        float kt[4], bk[4], bv[4], qg[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int i = 16 * I + rbq + w;
+            const bool live = kFull || i < p.len;
+            const uint32_t ob = p.swb[w] + i * 128;  // (i, c) in the bf16 staging tiles
+            float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK + ob));
+            float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ + ob));
+            float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + p.vbox + (ob - p.vblk)));
+            if (PRO) { kv *= s_rn[i]; qv *= s_rn[64 + i]; }
+            if (!live) { kv = 0.f; qv = 0.f; vv = 0.f; }
+            const float b = p.s_beta[i];
+            const float gi = p.g[I][w];
+            float dc, F, Gm, rowf;
+            if (!st) {
+                dc = __expf(p.anc[I] - gi);  // e^{a_I - g_i} in [e^-40, e^40]
+                rowf = recip_approx(dc);     // e^{g_i - a_I}
+                F = dc * tau;                // >= e^-80: a normal float
+                Gm = rowf * ea;              // e^{g_i} (only values below e^-47 lose digits)
+            } else {
+                dc = 0.f;                    // left to the exact per-element terms
+                rowf = 0.f;
+                F = __expf(p.gl[I] - gi);
+                Gm = __expf(gi);
+            }
+            *reinterpret_cast<float*>(sm + OFF_G + p.colf + i * 128 + p.swf[w]) = p.any_strong ? gi : rowf;
+            // column tiles: (n, c) at q4 * 160 * 128 + n * 128 + swizzle, n = y_row(R) + i = i mod 8
+            unsigned char* ycol = sm + OFF_Y + q4 * 20480 + p.swf[w] + i * 128;
+            const float kf = kv * F;
+            *reinterpret_cast<float*>(ycol + y_row(I) * 128) = to_tf32_op(kv * dc);
+#pragma unroll
+            for (int R = I + 1; R < 4; ++R) *reinterpret_cast<float*>(ycol + y_row(R) * 128) = to_tf32_op(kf * rho[R]);
+            kt[w] = to_tf32_op(kf * kap);
+            bk[w] = to_tf32_op(b * kv * Gm);
+            bv[w] = to_tf32_op(b * vv);
+            qg[w] = qv * Gm;
+        }
+        *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+        tmem_st4(p.tq + TM_BK + 16 * I + rbq, bk);
+        tmem_st4(p.tq + TM_BV + 16 * I + rbq, bv);
+        tmem_st4(p.tq + TM_QG + 16 * I + rbq, qg);
+    }
+}
+
 // SG: Gated DeltaNet gates -- log_alpha is [T_total, H], one decay rate per token and head, read
 // with beta and broadcast over the key channels (tm_g is then unused).
 // PRO: q and k arrive raw; every use of a row is scaled by 1 / its L2 norm, computed per chunk.
@@ -610,62 +690,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // kSpanLimit over it (every factor is then <= e^{kSpanLimit / 2}); else four 16-row blocks
         const bool one = *s_wide == 0u;
 
-        // ---- 3: per element (row i, channel c): the row factor e^{g_i - a} (for the row pass; g itself when
-        //      some channel decays strongly), the column tiles of MMA 1, Kt^T (MMAs 3-4), (beta K e^G)^T,
-        //      (beta V)^T (MMA 2) and (Q e^G)^T.  For i in block I, F_i = e^{g_eI - g_i} <= 1 (eI the block's
-        //      last row); diagonal column factor e^{a_I - g_i} (1 / the row factor); column factor of a later
-        //      block R: e^{a_R - g_eI} F_i (both <= 1)
-        auto elementwise = [&](auto full_chunk) {
-            constexpr bool kFull = decltype(full_chunk)::value;  // every row live: no masks
-#pragma unroll
-            for (int I = 0; I < 4; ++I) {
-                const bool st = (strong >> I) & 1u;
-                const float tau = f_tau[I * 128 + c], kap = f_kap[I * 128 + c], ea = f_ea[I * 128 + c];
-                float rho[4];
-#pragma unroll
-                for (int R = I + 1; R < 4; ++R) rho[R] = f_rho[rho_idx(R, I) * 128 + c];
-                float kt[4], bk[4], bv[4], qg[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const int i = 16 * I + rbq + w;
-                    const bool live = kFull || i < len;
-                    const uint32_t ob = swb[w] + i * 128;  // (i, c) in the bf16 staging tiles
-                    float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SK + ob));
-                    float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_SQ + ob));
-                    float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + vbox + (ob - vblk)));
-                    if (PRO) { kv *= s_rn[i]; qv *= s_rn[64 + i]; }
-                    if (!live) { kv = 0.f; qv = 0.f; vv = 0.f; }
-                    const float b = s_beta[i];
-                    float dc, F, Gm, rowf;
-                    if (!st) {
-                        dc = __expf(anc[I] - g[I][w]);  // e^{a_I - g_i} in [e^-40, e^40]
-                        rowf = recip_approx(dc);        // e^{g_i - a_I}
-                        F = dc * tau;                   // >= e^-80: a normal float
-                        Gm = rowf * ea;                 // e^{g_i} (only values below e^-47 lose digits)
-                    } else {
-                        dc = 0.f;                       // left to the exact per-element terms
-                        rowf = 0.f;
-                        F = __expf(gl[I] - g[I][w]);
-                        Gm = __expf(g[I][w]);
-                    }
-                    *reinterpret_cast<float*>(sm + OFF_G + colf + i * 128 + swf[w]) = any_strong ? g[I][w] : rowf;
-                    // column tiles: (n, c) at q4 * 160 * 128 + n * 128 + swizzle, n = y_row(R) + i = i mod 8
-                    unsigned char* ycol = sm + OFF_Y + q4 * 20480 + swf[w] + i * 128;
-                    const float kf = kv * F;
-                    *reinterpret_cast<float*>(ycol + y_row(I) * 128) = to_tf32_op(kv * dc);
-#pragma unroll
-                    for (int R = I + 1; R < 4; ++R) *reinterpret_cast<float*>(ycol + y_row(R) * 128) = to_tf32_op(kf * rho[R]);
-                    kt[w] = to_tf32_op(kf * kap);
-                    bk[w] = to_tf32_op(b * kv * Gm);
-                    bv[w] = to_tf32_op(b * vv);
-                    qg[w] = qv * Gm;
-                }
-                *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
-                tmem_st4(tq + TM_BK + 16 * I + rbq, bk);
-                tmem_st4(tq + TM_BV + 16 * I + rbq, bv);
-                tmem_st4(tq + TM_QG + 16 * I + rbq, qg);
-            }
-        };
+        // ---- 3: per element (row i, channel c), the operands of MMAs 1 to 4 (the four-block pass is
+        //      elementwise_blocks)
         // one anchor: per element the factor e^{a - g_i} (<= e^{kSpanLimit / 2} either way) and its
         // reciprocal give both MMA 1 operands straight from the element: rows i and 64 + i of
         // X = [K; Q] e^{G - a}, row i of Y = K e^{a - G}; then Kt^T = (K e^{a - G})^T e^{g_C - a},
@@ -712,8 +738,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (len == C) elementwise_one(std::true_type{});
             else elementwise_one(std::false_type{});
         } else {
-            if (len == C) elementwise(std::true_type{});
-            else elementwise(std::false_type{});
+            BlockPass bp;
+#pragma unroll
+            for (int I = 0; I < 4; ++I) {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) bp.g[I][w] = g[I][w];
+                bp.anc[I] = anc[I];
+                bp.gl[I] = gl[I];
+                bp.swf[I] = swf[I];
+                bp.swb[I] = swb[I];
+            }
+            bp.s_beta = s_beta;
+            bp.strong = strong;
+            bp.tq = tq;
+            bp.colf = colf;
+            bp.vbox = vbox;
+            bp.vblk = vblk;
+            bp.len = len;
+            bp.any_strong = any_strong;
+            if (len == C) elementwise_blocks<PRO, true>(bp);
+            else elementwise_blocks<PRO, false>(bp);
             __syncthreads();
         }
 
