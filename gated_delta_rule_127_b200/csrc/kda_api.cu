@@ -1,13 +1,23 @@
 // kda_api.cu -- the C ABI of libkda: host-side validation, dispatch to the kernels, status words.
 //
 // Nothing here computes any part of the operator; it checks arguments, picks the kernel and
-// launches it on the caller's stream.
+// launches it on the caller's stream.  Each call's launches sit in an NVTX range named for the entry
+// point and the path taken (header-only NVTX: free unless a profiler is attached).
+//
+// Built with -DKDA_DEBUG (libkda_debug.so), chunk_fwd also copies cu_seqlens to the host, waiting
+// on the caller's stream, and checks the sequence boundaries and the chunk-slot work list against
+// the workspace before any launch: a malformed batch then returns KDA_ERR_INVALID_ARG instead of
+// setting KDA_DEVFLAG_CU_SEQLENS on the device.
 #include <atomic>
 #include <mutex>
+#include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "kda.h"
 #include "kda_internal.h"
 #include "kda_testing.h"
+#include "kda_wy.cuh"
 
 namespace kda {
 
@@ -44,6 +54,35 @@ bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p
 bool valid_dtype(kda_dtype d) { return d == KDA_BF16 || d == KDA_FP32; }
 size_t dtype_size(kda_dtype d) { return d == KDA_FP32 ? 4 : 2; }
 bool supported_dim(int d) { return d == 64 || d == 128; }
+
+// NVTX range for the lifetime of a call's launches.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+
+#ifdef KDA_DEBUG
+// Host-side checks of a packed batch (debug builds): boundaries from 0 to T_total, not decreasing,
+// and every sequence's chunks inside the chunk-slot range the workspace was sized for.
+kda_status debug_check_batch(const int32_t* cu_seqlens, int64_t T_total, int N, void* stream) {
+    if (!cu_seqlens) return KDA_OK;
+    std::vector<int32_t> cu(static_cast<size_t>(N) + 1);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(cu.data(), cu_seqlens, cu.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cu[0] != 0 || cu[N] != T_total) return KDA_ERR_INVALID_ARG;
+    const int64_t slots = wy::num_slots(T_total, N);
+    for (int n = 0; n < N; ++n) {
+        if (cu[n + 1] < cu[n]) return KDA_ERR_INVALID_ARG;
+        const int64_t chunks = (static_cast<int64_t>(cu[n + 1]) - cu[n] + wy::C - 1) / wy::C;
+        if (wy::slot_base(cu[n], n) + chunks > slots) return KDA_ERR_INVALID_ARG;
+        if (n + 1 < N && wy::slot_base(cu[n], n) + chunks > wy::slot_base(cu[n + 1], n + 1))
+            return KDA_ERR_INVALID_ARG;  // two sequences' records would share a slot
+    }
+    return KDA_OK;
+}
+#endif
 
 }  // namespace
 
@@ -105,10 +144,15 @@ kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* lo
     a.out_gate = out_gate; a.norm_weight = norm_weight; a.norm_eps = norm_eps;
     a.wait_polls = consumer_wait_polls();
     if (device_flags_ptr(&a.flags) != cudaSuccess) return KDA_ERR_CUDA;
+#ifdef KDA_DEBUG
+    if (const kda_status st = debug_check_batch(cu_seqlens, T_total, N, stream); st != KDA_OK) return st;
+#endif
 
     cudaError_t err;
     bool epilogue_fused = false;
-    if (chunk_tc_path(a.T_total, a.dtype_qkv, a.dk, a.dv) && have_ws && need > 0) {
+    const bool tc = chunk_tc_path(a.T_total, a.dtype_qkv, a.dk, a.dv) && have_ws && need > 0;
+    NvtxRange range(tc ? "kda_chunk_fwd: tensor-core path" : "kda_chunk_fwd: CUDA-core path");
+    if (tc) {
         err = launch_chunk_prep(a);
         if (err == cudaSuccess) err = launch_chunk_scan(a);  // the scan applies the epilogue itself
         epilogue_fused = true;
@@ -150,6 +194,7 @@ kda_status decode_step(const void* q, const void* k, const void* v, const void* 
     a.beta_logits = (options & KDA_OPT_BETA_LOGITS) != 0;
     a.epilogue = (options & KDA_OPT_OUTPUT_NORM_GATE) != 0;
     a.out_gate = out_gate; a.norm_weight = norm_weight; a.norm_eps = norm_eps;
+    NvtxRange range("kda_decode_step");
     return launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -13,7 +13,8 @@ from typing import Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkda.so")
+# KDA_DEBUG=1 selects the debug build (host-side checks of packed batches before any launch)
+LIB_PATH = os.path.join(_HERE, "libkda_debug.so" if os.environ.get("KDA_DEBUG") == "1" else "libkda.so")
 INCLUDE_DIR = os.path.join(os.path.dirname(_HERE), "include")
 HEADER_PATH = os.path.join(INCLUDE_DIR, "kda.h")
 

@@ -26,6 +26,13 @@ def test_every_declared_symbol_is_exported(lib):
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
 
 
+def test_debug_build_exports_the_same_symbols(lib):
+    # the KDA_DEBUG=1 build differs only in host-side checks of packed batches
+    dbg = ctypes.CDLL(kbuild.LIB_DEBUG)
+    for name in kda.header_symbols():
+        assert ctypes.cast(getattr(dbg, name), ctypes.c_void_p).value, name
+
+
 def test_wait_limit_hook_needs_no_device(lib):
     # the test hook only sets a process-wide number; restore the default afterwards
     kda.kda_testing_set_wait_limit(0)
