@@ -144,7 +144,7 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: 
     cu_seqlens [N+1] int32 CUDA tensor, or None with `num_seqs` equal-length sequences (default 1).
     Returns (o [T, H, dv], final_state [N, H, dk, dv] fp32 or None).
     A workspace of kda_chunk_fwd_workspace_size bytes is allocated when none is given; with
-    use_workspace=False none is passed and the library runs its workspace-free kernel.
+    use_workspace=False none is passed and the library runs its CUDA-core path.
     """
     return _chunk_fwd("kda_chunk_fwd", q, k, v, log_alpha, beta, initial_state, cu_seqlens, num_seqs, chunk_size,
                       o, final_state, output_final_state, dtype_o, workspace, use_workspace, stream)

@@ -43,12 +43,14 @@ def _check_full(inp, dtype, use_workspace=True):
 
 def test_tiny_fp32_workload():
     inp = gen.make_workload("tiny_fp32", device=DEV)
-    _check_full(inp, torch.float32)
+    eo, es = _check_full(inp, torch.float32)
+    print(f"\ntiny_fp32: o_err {eo:.3e}, state_err {es:.3e} (every unit)")
 
 
 def test_prefill_b2_h4_t2048_workload():
     inp = gen.make_workload("prefill_b2_h4_t2048", device=DEV)
-    _check_full(inp, torch.bfloat16)
+    eo, es = _check_full(inp, torch.bfloat16)
+    print(f"\nprefill_b2_h4_t2048: o_err {eo:.3e}, state_err {es:.3e} (every unit)")
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
