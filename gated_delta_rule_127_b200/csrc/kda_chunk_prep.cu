@@ -147,9 +147,10 @@ constexpr uint32_t TM_BV = 384;   // (beta V)^T, 128 (dv) x 64 (s), A of MMA 2
 constexpr uint32_t TM_QG = 448;   // (Q e^G)^T, 128 (j) x 64 (t): copied into MMA 3's accumulator before it runs
 constexpr uint32_t TM_WT = 0;     // W^T, 128 x 64 (after MMA 1)
 constexpr uint32_t TM_UT = 64;    // U^T, 128 x 64
-constexpr uint32_t TM_DW = 0;     // MMA 3, 128 (j) x 256, seeded [Diag(e^{g_C}) | (Q e^G)^T | 0]: Mt^T, then Qh^T in
-                                  //   two parts (P_hi, P_lo)                                   (after MMA 2)
-constexpr uint32_t TM_DU = 256;   // MMA 4, 128 (dv) x 256: B^T, then Uo^T in two parts (P_hi, P_lo)
+constexpr uint32_t TM_DU = 0;     // MMA 4, 128 (dv) x 256: B^T, then Uo^T in two parts (P_hi, P_lo)  (after MMA 2)
+constexpr uint32_t TM_DW = 256;   // MMA 3, 128 (j) x 256, seeded [Diag(e^{g_C}) | (Q e^G)^T | 0]: Mt^T, then Qh^T in
+                                  //   two parts.  Over the dead MMA 2 operands: each thread seeds it right after
+                                  //   reading its own (Q e^G)^T columns, which the seed's zero part then covers
 constexpr uint32_t TM_COLS = 512;
 
 // Byte offset of element (t, i) of the fp32 P tile at OFF_PF: rows of 256 bytes, 16-byte chunk i / 4
@@ -1000,39 +1001,39 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         failed = !mbar_wait(bar_m2, par, wait_polls);
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
-        uint32_t qg[16];  // (Q e^G)^T of lane c, tokens 16 qr .. +15: moved into MMA 3's accumulator below
-        {   // W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..)
-            uint32_t x[32];
+        {   // W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..);
+            // MMA 3's accumulator <- [Diag(e^{g_C}) | (Q e^G)^T | 0] (lane j = c; the MMA then adds -W^T [Kt; P]^T).
+            // The seed lands on dead columns (MMA 1's accumulator and MMA 2's operands) and on this thread's own
+            // (Q e^G)^T columns, read just before: no other thread's pending read is overwritten.
+            uint32_t x[32], qg[16];
             const bool isw = qr < 2;
             tmem_ld32_nw(tq + (isw ? TM_WT : TM_UT) + 32 * (qr & 1), x);
             tmem_ld16_nw(tq + TM_QG + 16 * qr, qg);
             tmem_ld_wait();
             after_ld_wait(x);
             after_ld_wait(qg);
+            static_assert(TM_DW + 192 == TM_QG && TM_DW >= TM_D1 && TM_DU + 256 <= TM_DW, "seed placement");
+            {
+                float d[32];
+                const float gam = s_gam[c];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) d[e] = (32 * qr + e == c) ? gam : 0.f;
+                tmem_st32(tq + TM_DW + 32 * qr, d);
+                float qf[16], z[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    qf[e] = __uint_as_float(qg[e]);
+                    z[e] = 0.f;
+                }
+                tmem_st16(tq + TM_DW + 128 + 16 * qr, qf);
+                tmem_st16(tq + TM_DW + 192 + 16 * qr, z);
+            }
             unsigned char* tile = sm + (isw ? OFF_WT : OFF_UT);
             auto r = [&](int e) { return to_tf32_op(__uint_as_float(x[e])); };
 #pragma unroll
             for (int e4 = 0; e4 < 32; e4 += 4)
                 *reinterpret_cast<float4*>(tile + sw128_off(c, 32 * (qr & 1) + e4, 128)) =
                     make_float4(r(e4), r(e4 + 1), r(e4 + 2), r(e4 + 3));
-        }
-        tc_fence_before_sync();
-        __syncthreads();  // W^T, U^T and (Q e^G)^T are read: MMA 3's accumulator may be filled over them
-        tc_fence_after_sync();
-        {   // MMA 3's accumulator <- [Diag(e^{g_C}) | (Q e^G)^T | 0] (lane j = c): the MMA then adds -W^T [Kt; P]^T
-            float d[32];
-            const float gam = s_gam[c];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) d[e] = (32 * qr + e == c) ? gam : 0.f;
-            tmem_st32(tq + TM_DW + 32 * qr, d);
-            float qf[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) qf[e] = __uint_as_float(qg[e]);
-            tmem_st16(tq + TM_DW + 128 + 16 * qr, qf);
-            float z[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) z[e] = 0.f;
-            tmem_st16(tq + TM_DW + 192 + 16 * qr, z);
             tmem_st_wait();
         }
         fence_async_smem();
