@@ -286,7 +286,7 @@ __device__ __forceinline__ void warp_store_16x8(float* z, int zs, const float (&
 }
 
 // T = (I + A)^{-1} for A strictly lower (fp32, row stride TP) into tm, the part on and below the
-// diagonal blocks (zero_above_blocks writes the rest); xs: 1024 floats of scratch.  Run by four warps,
+// diagonal blocks (the zeros above them go straight into the operand tile); xs: 1024 floats of scratch.  Run by four warps,
 // iw = 0..3 their index, joined by named barrier 1.  The 16 x 16 diagonal blocks by forward
 // substitution in fp32, then two merges of [[T1, 0], [T21, T2]] with T21 = -T2 (A21 T1): 16 -> 32 (both
 // halves at once) and 32 -> 64.  Their products run as 16 x 8 tiles on the warps' tensor cores with tf32
@@ -349,13 +349,21 @@ __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, f
         warp_store_16x8(tm + 48 * TP + 8 * ct, TP, d, true);
     }
 }
-// The zeros of T above its diagonal blocks (rows r, columns 16 (r / 16 + 1) .. 63), by 128 threads
-// (t = 0..127), four at a time.
-__device__ __forceinline__ void zero_above_blocks(float* tm, int t) {
+// T's tf32 operand tile for MMA 2 (K-major rows r x K s, sw128_off(r, s, 64)), by 128 threads (t = 0..127),
+// four elements at a time: lower = true takes the part on and below the diagonal blocks from tm (fp32, row
+// stride TP), lower = false writes the zeros above them.
+__device__ __forceinline__ void t_operand_tile(const float* tm, unsigned char* timg, int t, bool lower) {
 #pragma unroll
     for (int e = t; e < 64 * 16; e += 128) {
         const int r = e >> 4, c4 = (e & 15) * 4;
-        if (c4 >= 16 * ((r >> 4) + 1)) *reinterpret_cast<float4*>(tm + r * TP + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool below = c4 < 16 * ((r >> 4) + 1);
+        if (below != lower) continue;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lower) {
+            const float4 x = *reinterpret_cast<const float4*>(tm + r * TP + c4);
+            v = make_float4(to_tf32_op(x.x), to_tf32_op(x.y), to_tf32_op(x.z), to_tf32_op(x.w));
+        }
+        *reinterpret_cast<float4*>(timg + sw128_off(r, c4, 64)) = v;
     }
 }
 
@@ -596,8 +604,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const float* s_beta = s_beta2 + 64 * par;
         cur_par = par;
         mma_issued = 0;
-        failed = !mbar_wait(bar_tma, par, wait_polls);
-        if (__syncthreads_or(failed)) { failed = true; break; }
+        failed = !mbar_wait(bar_tma, par, wait_polls);  // acted on at the barrier that ends step 1
         tc_fence_after_sync();
 
         // ---- elementwise pass, 1: log-decays of channel c over rows 16 I + rbq .. + 3 of each block I; the
@@ -637,7 +644,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (lane == 0) s_rn[row] = inv_norm(ss);
             }
         }
-        __syncthreads();
+        if (__syncthreads_or(failed)) { failed = true; break; }
         // ---- 2: g from the chunk start; every block's first and last g, anchor and strong-decay flag for
         //      channel c (the four threads of a channel compute the same; those with qr = 0 publish them)
         float anc[4], gl[4];
@@ -948,13 +955,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (lane == 0 && warp < kLoads && tn.id >= 0) load_box(tn, warp);
         load_beta(tn, par ^ 1u);
 
-        // ---- T = (I + A)^{-1} by warps 0, 1, 4, 5 (A-lane warps), the zeros above its diagonal blocks by
-        //      warps 8, 9, 12, 13; meanwhile, for one-anchor chunks, the P-lane warps move P into [Kt; P].
-        //      Then T's tf32 operand tile.
+        // ---- T = (I + A)^{-1} by warps 0, 1, 4, 5 (A-lane warps), the zeros of its tf32 operand tile above the
+        //      diagonal blocks by warps 8, 9, 12, 13; meanwhile, for one-anchor chunks, the P-lane warps move
+        //      P into [Kt; P].  Then T's operand tile by all threads.
         if (q4 < 2) {
+            const int iw = (warp & 1) | (((warp >> 2) & 1) << 1);  // 0..3 within each group of four warps
             if (warp < 8) unit_lower_inverse(reinterpret_cast<const float*>(sm + OFF_A), reinterpret_cast<float*>(sm + OFF_T32),
-                                             xs, (warp & 1) | ((warp >> 2) << 1));
-            else zero_above_blocks(reinterpret_cast<float*>(sm + OFF_T32), (tid & 31) | (((warp & 1) | (((warp >> 2) - 2) << 1)) << 5));
+                                             xs, iw);
+            else t_operand_tile(nullptr, sm + OFF_TIMG, (tid & 31) | (iw << 5), false);
         } else if (one) {  // lane rows 64..127: P (lower with the diagonal), columns 16 qr ..
             const int row = c & 63, i0 = 16 * qr;
             float x[16];
@@ -968,14 +976,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
         __syncthreads();
-        {
+        {   // the part of T's operand tile on and below the diagonal blocks, four elements a thread at a time
             const float* t32 = reinterpret_cast<const float*>(sm + OFF_T32);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int idx = tid + THREADS * u;
-                const int r = idx >> 4, s4 = (idx & 15) * 4;
-                const float4 t = *reinterpret_cast<const float4*>(t32 + r * TP + s4);
-                *reinterpret_cast<float4*>(sm + OFF_TIMG + sw128_off(r, s4, 64)) =
+            for (int e = tid; e < 64 * 16; e += THREADS) {
+                const int r = e >> 4, c4 = (e & 15) * 4;
+                if (c4 >= 16 * ((r >> 4) + 1)) continue;
+                const float4 t = *reinterpret_cast<const float4*>(t32 + r * TP + c4);
+                *reinterpret_cast<float4*>(sm + OFF_TIMG + sw128_off(r, c4, 64)) =
                     make_float4(to_tf32_op(t.x), to_tf32_op(t.y), to_tf32_op(t.z), to_tf32_op(t.w));
             }
         }
@@ -998,8 +1006,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mma_issued |= 2u;
         }
         if (tid == kWalker) slots[aft] = walker->next();  // while MMA 2 runs: the task after the next
-        failed = !mbar_wait(bar_m2, par, wait_polls);
-        if (__syncthreads_or(failed)) { failed = true; break; }
+        failed = !mbar_wait(bar_m2, par, wait_polls);  // acted on at the barrier after the read-out
         tc_fence_after_sync();
         {   // W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..);
             // MMA 3's accumulator <- [Diag(e^{g_C}) | (Q e^G)^T | 0] (lane j = c; the MMA then adds -W^T [Kt; P]^T).
@@ -1038,7 +1045,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         fence_async_smem();
         tc_fence_before_sync();
-        __syncthreads();
+        if (__syncthreads_or(failed)) { failed = true; break; }
 
         // ---- MMA 3: [Diag(e^{g_C}) | (Q e^G)^T | 0] - W^T [Kt; P_hi; P_lo]^T = [Mt | Qh^T split in two halves];
         //      MMA 4: U^T [Kt; P_hi; P_lo]^T = [B^T | Uo^T split in two halves].  M=128, N=256, K=64 (tokens s);
