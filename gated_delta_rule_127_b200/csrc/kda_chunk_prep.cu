@@ -136,20 +136,15 @@ static_assert(OFF_TIMG % 1024 == 0 && OFF_WT % 1024 == 0 && OFF_UT % 1024 == 0 &
 
 // first row of column tile R within the 160-row tile (tile R has 16 R + 16 rows)
 __host__ __device__ constexpr int y_row(int R) { return 8 * R * (R + 1); }
-// Tensor-memory column of token s in the MMA 2 operands (beta K e^G)^T, (beta V)^T and in (Q e^G)^T: the
-// token's 4-row group (s / 4) % 4 and its 16-row block s / 16 swapped, so that the 16 rows 16 I + 4 q + w
-// (I, w = 0..3) of an elementwise thread with group q are 16 adjacent columns, written by one store per
-// operand.  MMA 2 contracts over s, so T's operand tile takes its K index in the same order.
-__host__ __device__ constexpr int tcol(int s) { return 16 * ((s >> 2) & 3) + 4 * (s >> 4) + (s & 3); }
 // index of the block pair (R, I), R > I, in OFF_RHO
 __host__ __device__ constexpr int rho_idx(int R, int I) { return R * (R - 1) / 2 + I; }
 
 // ---- tensor memory columns (512 allocated)
 constexpr uint32_t TM_X = 0;      // [K; Q] rows scaled by e^{G - a}, 128 x 128, A of MMA 1
 constexpr uint32_t TM_D1 = 128;   // MMA 1, 128 x 160: block R's columns at TM_D1 + y_row(R)
-constexpr uint32_t TM_BK = 320;   // (beta K e^G)^T, 128 (c) x 64 (s at column tcol(s)), A of MMA 2
-constexpr uint32_t TM_BV = 384;   // (beta V)^T, 128 (dv) x 64 (s at tcol(s)), A of MMA 2
-constexpr uint32_t TM_QG = 448;   // (Q e^G)^T, 128 (j) x 64 (t at tcol(t)): copied into MMA 3's accumulator
+constexpr uint32_t TM_BK = 320;   // (beta K e^G)^T, 128 (c) x 64 (s), A of MMA 2
+constexpr uint32_t TM_BV = 384;   // (beta V)^T, 128 (dv) x 64 (s), A of MMA 2
+constexpr uint32_t TM_QG = 448;   // (Q e^G)^T, 128 (j) x 64 (t): copied into MMA 3's accumulator
 constexpr uint32_t TM_WT = 0;     // W^T, 128 x 64 (after MMA 1)
 constexpr uint32_t TM_UT = 64;    // U^T, 128 x 64
 constexpr uint32_t TM_DU = 0;     // MMA 4, 128 (dv) x 256: B^T, then Uo^T in two parts (P_hi, P_lo)  (after MMA 2)
@@ -354,7 +349,7 @@ __device__ __forceinline__ void unit_lower_inverse(const float* am, float* tm, f
         warp_store_16x8(tm + 48 * TP + 8 * ct, TP, d, true);
     }
 }
-// T's tf32 operand tile for MMA 2 (K-major rows r x K s, sw128_off(r, tcol(s), 64)), by 128 threads (t = 0..127),
+// T's tf32 operand tile for MMA 2 (K-major rows r x K s, sw128_off(r, s, 64)), by 128 threads (t = 0..127),
 // four elements at a time: lower = true takes the part on and below the diagonal blocks from tm (fp32, row
 // stride TP), lower = false writes the zeros above them.
 __device__ __forceinline__ void t_operand_tile(const float* tm, unsigned char* timg, int t, bool lower) {
@@ -368,7 +363,7 @@ __device__ __forceinline__ void t_operand_tile(const float* tm, unsigned char* t
             const float4 x = *reinterpret_cast<const float4*>(tm + r * TP + c4);
             v = make_float4(to_tf32_op(x.x), to_tf32_op(x.y), to_tf32_op(x.z), to_tf32_op(x.w));
         }
-        *reinterpret_cast<float4*>(timg + sw128_off(r, tcol(c4), 64)) = v;  // K index in tcol order
+        *reinterpret_cast<float4*>(timg + sw128_off(r, c4, 64)) = v;
     }
 }
 
@@ -446,9 +441,9 @@ __device__ __noinline__ void elementwise_blocks(const BlockPass& p) {
             qg[w] = qv * Gm;
         }
         *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
-        tmem_st4(p.tq + TM_BK + tcol(16 * I + rbq), bk);  // (the four rows' columns are adjacent)
-        tmem_st4(p.tq + TM_BV + tcol(16 * I + rbq), bv);
-        tmem_st4(p.tq + TM_QG + tcol(16 * I + rbq), qg);
+        tmem_st4(p.tq + TM_BK + 16 * I + rbq, bk);
+        tmem_st4(p.tq + TM_BV + 16 * I + rbq, bv);
+        tmem_st4(p.tq + TM_QG + 16 * I + rbq, qg);
     }
 }
 
@@ -716,10 +711,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             unsigned char* xcol = sm + OFF_XF + q4 * 16384;  // K-block of channel c
             unsigned char* ycol = sm + OFF_YF + q4 * 8192;
 #pragma unroll
-            float bk[16], bv[16], qg[16];  // columns tcol(16 I + rbq + w) = 16 qr + 4 I + w: index 4 I + w
-#pragma unroll
             for (int I = 0; I < 4; ++I) {
-                float kt[4];
+                float kt[4], bk[4], bv[4], qg[4];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
                     const int i = 16 * I + rbq + w;
@@ -740,16 +733,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     *reinterpret_cast<float*>(xcol + 8192 + o) = to_tf32_op(qv * rowf);  // row 64 + i
                     const float Gm = rowf * ea;
                     kt[w] = to_tf32_op(ky * kap);
-                    bk[4 * I + w] = to_tf32_op(b * kv * Gm);
-                    bv[4 * I + w] = to_tf32_op(b * vv);
-                    qg[4 * I + w] = qv * Gm;
+                    bk[w] = to_tf32_op(b * kv * Gm);
+                    bv[w] = to_tf32_op(b * vv);
+                    qg[w] = qv * Gm;
                 }
                 *reinterpret_cast<float4*>(sm + OFF_KP + sw128_off(c, 16 * I + rbq, 256)) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+                tmem_st4(tq + TM_BK + 16 * I + rbq, bk);
+                tmem_st4(tq + TM_BV + 16 * I + rbq, bv);
+                tmem_st4(tq + TM_QG + 16 * I + rbq, qg);
             }
-            static_assert(tcol(4) == 16 && tcol(16) == 4, "column order");
-            tmem_st16(tq + TM_BK + 16 * qr, bk);
-            tmem_st16(tq + TM_BV + 16 * qr, bv);
-            tmem_st16(tq + TM_QG + 16 * qr, qg);
         };
         if (one) {
             if (len == C) elementwise_one(std::true_type{});
@@ -993,7 +985,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int r = e >> 4, c4 = (e & 15) * 4;
                 if (c4 >= 16 * ((r >> 4) + 1)) continue;
                 const float4 t = *reinterpret_cast<const float4*>(t32 + r * TP + c4);
-                *reinterpret_cast<float4*>(sm + OFF_TIMG + sw128_off(r, tcol(c4), 64)) =
+                *reinterpret_cast<float4*>(sm + OFF_TIMG + sw128_off(r, c4, 64)) =
                     make_float4(to_tf32_op(t.x), to_tf32_op(t.y), to_tf32_op(t.z), to_tf32_op(t.w));
             }
         }
@@ -1020,14 +1012,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_after_sync();
         {   // W^T and U^T, rounded to tf32, into their K-major operand tiles (row j = lane, K s = 32 (qr & 1) ..);
             // MMA 3's accumulator <- [Diag(e^{g_C}) | (Q e^G)^T | 0] (lane j = c; the MMA then adds -W^T [Kt; P]^T).
-            // The seed lands on dead columns (MMA 1's accumulator and MMA 2's operands) and on this thread's own
-            // (Q e^G)^T columns, read just before: no other thread's pending read is overwritten.
+            // The seed lands on dead columns (MMA 1's accumulator and MMA 2's operands) and, for its zero part,
+            // on exactly the (Q e^G)^T columns this thread has just read: no other thread's pending read is
+            // overwritten.
             uint32_t x[32], qg[16];
             const bool isw = qr < 2;
             tmem_ld32_nw(tq + (isw ? TM_WT : TM_UT) + 32 * (qr & 1), x);
-#pragma unroll
-            for (int g4 = 0; g4 < 4; ++g4)  // tokens 16 qr + 4 g4 .. + 3 sit at columns tcol(16 qr + 4 g4) ..
-                tmem_ld4_nw(tq + TM_QG + tcol(16 * qr + 4 * g4), qg + 4 * g4);
+            tmem_ld16_nw(tq + TM_QG + 16 * qr, qg);
             tmem_ld_wait();
             after_ld_wait(x);
             after_ld_wait(qg);
@@ -1045,7 +1036,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     z[e] = 0.f;
                 }
                 tmem_st16(tq + TM_DW + 128 + 16 * qr, qf);
-                tmem_st16(tq + TM_DW + 192 + 16 * qr, z);
+                tmem_st16(tq + TM_DW + 192 + 16 * qr, z);  // (over the (Q e^G)^T columns just read)
             }
             unsigned char* tile = sm + (isw ? OFF_WT : OFF_UT);
             auto r = [&](int e) { return to_tf32_op(__uint_as_float(x[e])); };
