@@ -187,11 +187,37 @@ def measured_peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """CUDA/C++ source without its comments and blank space, so that a comment edit does not count as
+    a kernel change (string literals holding comment markers are kept whole)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        ch = text[i]
+        if ch == '"':  # string literal
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(ch)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def sources_digest(paths):
+    """Digest of the kernels' code (comments and spacing excluded), matched against the one stored
+    with the profiled traffic."""
     h = hashlib.sha256()
     for p in paths:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -19,15 +19,20 @@
 // the two halves of each output product are summed when read out.  This removes the largest rounding
 // term of the outputs (P rounded to tf32), about a third of their largest error.
 // Everything is formed transposed, with the key channel (or value column) as the tensor-memory lane:
-// the elementwise pass owns a channel and writes its operands straight into tensor memory, and each
+// the elementwise pass owns a channel and writes MMA 2's operands straight into tensor memory, and each
 // record row goes from a lane's registers to the record in coalesced runs.  Every tcgen05 tf32 MMA
 // instruction costs about the same time for any N up to 192 (N = 256 about a third more), so the
 // products are grouped into few wide instructions: 16 for MMA 1, 16 for MMA 2, 8 each for MMAs 3 and 4.
 //
 // Decay factors: secondary chunking.  "일반 DPLR보다 줄어든 연산량" on the same page notes that with a
 // decay per channel the intra-chunk division is numerically delicate (a factor e^{-g} overflows) and
-// points to the log domain with a second level of chunking.  Each chunk is cut into four 16-row
-// blocks; row block R has one anchor a_R per channel, and
+// points to the log domain with a second level of chunking.  The kernels never form e^{-g}: every
+// factor is taken against an anchor a per channel, e^{g_r - g_i} = e^{g_r - a} e^{a - g_i}.
+// One anchor: a chunk whose log-decay spans at most 80 nats in every channel takes the midpoint of
+// each channel's span as its anchor, so no factor exceeds e^40.  MMA 1 is then one MMA with N = 64:
+// [K; Q] e^{G - a} against K e^{a - G}, both written by the elementwise pass into shared memory.
+// Four blocks: any other chunk is cut into four 16-row blocks; row block R has one anchor a_R per
+// channel, and
 //   e^{g_r - g_i} = e^{g_r - a_R} e^{a_R - g_i}        for r in block R and i up to the block's last row.
 // For i in an earlier block both factors are <= 1 whatever the decay (a_R is at most g at the
 // block's first row, which is at most g_i).  Inside the block a_R is the midpoint of the channel's
@@ -36,13 +41,15 @@
 // at the block's first row instead, is left out of the block's diagonal 16 x 16 product, and its
 // diagonal terms are added one by one with the exact e^{g_r - g_i}.  No factor exceeds e^40 and
 // every factor that underflows multiplies a true value at least as small, so every chunk is exact up
-// to rounding for every alpha in (0, 1).  MMA 1 is one MMA with N = 160: the [K; Q] rows scaled by
-// e^{G - a} (A operand in tensor memory) against the column tiles K e^{a_R - G} of all four blocks
-// stacked (16 + 32 + 48 + 64 rows); row r of block R keeps the columns of tile R.
+// to rounding for every alpha in (0, 1).  MMA 1 is then one MMA with N = 160: the [K; Q] rows scaled
+// by e^{G - a} (A operand in tensor memory, written by a row pass) against the column tiles
+// K e^{a_R - G} of all four blocks stacked (16 + 32 + 48 + 64 rows); row r of block R keeps the
+// columns of tile R.  The four-block elementwise pass is out of line (elementwise_blocks), so that
+// the kernel's registers are allocated for the one-anchor pass.
 //
 // Persistent CTAs of 512 threads, one per SM, each taking (chunk slot, head) tasks in turn; the next
 // task's input tiles are loaded while the current task runs its inverse and products, and the
-// record's Mt and Qh tiles leave through bulk copies while the next task starts.  Elementwise pass:
+// record's Mt and Qh tiles leave through a bulk copy while the next task starts.  Elementwise pass:
 // thread t owns key channel c = 32 (w % 4) + lane (its tensor-memory lane, w = warp) and rows
 // 16 I + 4 (w / 4) .. + 3 of every block I (a cumulative sum over 4-row groups, completed through
 // shared memory).  Row pass and read-outs: the warp's lane quadrant gives the row (or channel),

@@ -42,3 +42,15 @@ def test_reference_arm_under_torchrun_prints_once():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = _json_lines(r.stdout)
     assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_traffic_digest_ignores_comments_only():
+    # roofline.traffic stays valid across comment edits of the kernel sources, and no longer once the
+    # code itself changes
+    import bench
+    a = 'int f() { return 1; } // one\n/* block\n comment */ const char* s = "a // b /* c";\n'
+    b = 'int f()  {\n  return 1;   }  // other words\nconst char* s = "a // b /* c";'
+    c = 'int f() { return 2; }\nconst char* s = "a // b /* c";'
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert '"a // b /* c"' in bench._code_only(a)
