@@ -81,7 +81,8 @@ using wy::DV;
 
 constexpr int THREADS = 512;
 constexpr int TP = 68;  // row stride (floats) of the fp32 A and T tiles (conflict-free MMA fragment reads)
-constexpr float kSpanLimit = 80.f;  // largest log-decay span of a 16-row block kept in its MMA product
+constexpr float kSpanLimit = 80.f;  // largest log-decay span kept in an MMA product: over the chunk for the
+                                    // one-anchor form, over a 16-row block for the four-block form
 constexpr uint32_t kWaitPolls = kDefaultWaitPolls;  // bound of the waits that drain work in flight
 
 // ---- shared memory (bytes from a 1024-aligned base)
@@ -124,7 +125,7 @@ constexpr uint32_t OFF_TIMG = OFF_Y + 35840;   // T K-major rows r x K s (64), B
 constexpr uint32_t OFF_XS = OFF_Y + 52224;     // 32 x 32 fp32 scratch for the inverse
 constexpr uint32_t OFF_PF = OFF_Y + 56320;     // P fp32 [64][64] (16-byte chunks XOR-swizzled by row)
 // after MMA 2:
-constexpr uint32_t OFF_WT = OFF_Y;             // -W^T K-major rows j x K s (64), A of MMA 3
+constexpr uint32_t OFF_WT = OFF_Y;             // W^T K-major rows j x K s (64), A of MMA 3 (negated by its descriptor)
 constexpr uint32_t OFF_UT = OFF_Y + 32768;     // U^T K-major rows dv x K s (64), A of MMA 4
 // after MMAs 3 and 4: the record's [Mt; Qh] tile, in the record's layout, for one bulk copy (clear of
 // what the next task writes before it waits for the copy -- the group sums and the block factors -- and
